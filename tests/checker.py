@@ -1,0 +1,71 @@
+"""Comparison rules between a GPU result and the float64 oracle.
+
+Tolerances (stated once, used by every parity test):
+
+* bf16 outputs (fp32 accumulate): max-abs error <= 1e-2 and mean-abs error
+  <= 1e-3.  A bf16 output cannot be closer to the exact value than half a
+  bf16 ulp, and for |x| >= 4 half an ulp is 0.0156 > 1e-2, so the max-abs
+  test is applied to the *excess* over half an ulp of the oracle's value:
+  max(0, |gpu - oracle| - ulp_bf16(oracle)/2) <= 1e-2.  The raw max-abs
+  error is reported next to it.  The mean-abs bound is applied raw.
+* fp32 outputs: max-abs error <= 1e-5 (raw).
+* integer outputs (counts, masks): bit-exact.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+
+BF16_MAX_ABS = 1e-2
+BF16_MEAN_ABS = 1e-3
+F32_MAX_ABS = 1e-5
+
+
+def bf16_half_ulp(x):
+    """Half the spacing of bf16 numbers at |x| (8 significant bits)."""
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(x > 0, x, 1.0)))
+    e = np.maximum(e, -126.0)
+    return np.where(x > 0, 2.0 ** (e - 8), 2.0 ** -134)
+
+
+@dataclasses.dataclass
+class Cmp:
+    ok: bool
+    max_abs: float
+    mean_abs: float
+    max_excess: float
+    n: int
+    rule: str
+
+    def __str__(self):
+        return (f"{self.rule}: ok={self.ok} max_abs={self.max_abs:.3e} "
+                f"max_excess={self.max_excess:.3e} mean_abs={self.mean_abs:.3e} n={self.n}")
+
+
+def compare(gpu, ref, kind="bf16", max_abs=None, mean_abs=None) -> Cmp:
+    """Compare arrays; ``kind`` is "bf16" (half-ulp excess rule) or "f32"."""
+    g = np.asarray(gpu, dtype=np.float64)
+    r = np.asarray(ref, dtype=np.float64)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    both_inf = np.isinf(g) & np.isinf(r) & (np.sign(g) == np.sign(r))
+    err = np.where(both_inf, 0.0, np.abs(g - r))
+    err = np.where(np.isnan(err), np.inf, err)
+    n = err.size
+    mx = float(err.max()) if n else 0.0
+    mean = float(err.mean()) if n else 0.0
+    if kind == "bf16":
+        lim = BF16_MAX_ABS if max_abs is None else max_abs
+        mlim = BF16_MEAN_ABS if mean_abs is None else mean_abs
+        excess = np.maximum(0.0, err - np.where(np.isfinite(r), bf16_half_ulp(r), 0.0))
+        mex = float(excess.max()) if n else 0.0
+        ok = mex <= lim and mean <= mlim
+        rule = f"bf16(excess<={lim:g}, mean<={mlim:g})"
+    else:
+        lim = F32_MAX_ABS if max_abs is None else max_abs
+        mex = mx
+        ok = mx <= lim and (mean_abs is None or mean <= mean_abs)
+        rule = f"f32(max<={lim:g})"
+    return Cmp(ok, mx, mean, mex, n, rule)
