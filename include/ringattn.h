@@ -1,0 +1,192 @@
+/*
+ * ringattn.h — C ABI of a B200 (sm_100a) implementation of Ring Attention's
+ * blockwise *exact* attention, with the P ring ranks virtual on one GPU.
+ *
+ * Method (pages describing Ring Attention, cited by title and section):
+ *  - "Ring Attention技术解析：突破大模型长上下文训练瓶颈" §2.2: the sequence is
+ *    cut into P blocks; devices form a ring; each device sends its key/value
+ *    block to the next device and receives the previous one's.
+ *  - "手把手拆解RingAttention：如何用分布式计算突破百万token长视频处理瓶颈" §1:
+ *    queries stay, keys/values travel, and global attention is kept complete
+ *    (complexity table, row "RingAttention").  So the result is exactly
+ *    full softmax attention; partials are combined by an online softmax
+ *    (running max, running sum, rescale) / log-sum-exp merge.
+ *  - "RingAttention核心功能全解析", 核心API调用 and 核心技术原理 1: the call
+ *    ringattention(xq, xk, xv, attention_bias, segment_ids, blockwise_kwargs=
+ *    {query_chunk_size, key_chunk_size, causal_block_size, policy}); the
+ *    policy "nothing_saveable" means the backward recomputes attention from
+ *    the inputs (here: from the saved log-sum-exp).
+ *
+ * Conventions for every entry point
+ *  - Tensors are described by ra_tensor: a pointer plus dtype, rank, shape
+ *    and strides in ELEMENTS.  Data pointers are DEVICE pointers unless a
+ *    parameter says "host".  The caller owns every buffer; the library never
+ *    allocates device memory and keeps no state besides one device-side
+ *    status word per device.
+ *  - q, k, v, o, dO, dq, dk, dv are [B, S, H, D] (batch, token, head, head
+ *    dim); the head dim must be contiguous (stride 1) and D in {64, 128}.
+ *    bf16 tensors additionally need 16-byte aligned base pointers and
+ *    strides whose byte size is a multiple of 16 (they are read by TMA).
+ *  - lse, m, l are fp32 [B, H, S] (any strides).  LSE is in natural-log
+ *    units; a query row with no visible key has o = 0 and lse = -inf.
+ *  - attention_bias: NULL or fp32 [B, S]: additive bias per KEY, broadcast
+ *    over heads and queries; -inf masks the key.
+ *  - segment_ids: NULL or int32 [B, S]: a key is visible only to queries
+ *    with the same id.
+ *  - Masking uses global token positions: with causal_block_size c >= 1,
+ *    key j is visible to query i iff floor(i/c) >= floor(j/c); c = 0 means
+ *    non-causal.  Softmax scale is 1/sqrt(D).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  A non-zero return means nothing was launched and
+ *    the outputs are unspecified.  No exception or exit crosses the ABI.
+ *  - Errors detected on the device (a bounded wait that ran out) are
+ *    recorded in the device status word; ra_get_device_status() reads it.
+ */
+#ifndef RINGATTN_H_
+#define RINGATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { RA_F32 = 0, RA_BF16 = 1, RA_I32 = 2 } ra_dtype;
+
+enum {
+  RA_OK = 0,
+  RA_ERR_NULL = 1,           /* a required pointer is NULL */
+  RA_ERR_DTYPE = 2,          /* dtype not allowed for this argument, or inputs disagree */
+  RA_ERR_SHAPE = 3,          /* rank or shape mismatch between arguments */
+  RA_ERR_STRIDE = 4,         /* head dim not contiguous, or TMA alignment rules violated */
+  RA_ERR_DIVISIBILITY = 5,   /* S % ring_size, (S/ring_size) % chunk, or a size < 1 */
+  RA_ERR_UNSUPPORTED = 6,    /* D not in {64,128}, ring_size > 64, or bf16 path on a non-sm_100 device */
+  RA_ERR_WORKSPACE = 7,      /* workspace NULL or smaller than ra_workspace_size() */
+  RA_ERR_CUDA = 8,           /* a CUDA runtime call failed (launch, attribute, tensor map) */
+  RA_ERR_DEVICE_TIMEOUT = 9, /* device-side bounded wait ran out (reported by ra_get_device_status) */
+  RA_ERR_ORDER = 10          /* ring_order is not a permutation of 0..ring_size-1 */
+};
+
+typedef struct {
+  void* data;         /* device pointer (see each entry point) */
+  int32_t dtype;      /* ra_dtype */
+  int32_t ndim;       /* number of valid entries in shape / stride */
+  int64_t shape[4];
+  int64_t stride[4];  /* in elements */
+} ra_tensor;
+
+#define RA_MAX_RING 64
+
+typedef struct {
+  /* blockwise_kwargs of "RingAttention核心功能全解析" 核心技术原理 1: chunk sizes
+   * group the hardware's 128-token tiles; each must be >= 1 and divide S /
+   * ring_size.  They do not change the (exact) result. */
+  int64_t query_chunk_size;
+  int64_t key_chunk_size;
+  /* 0 = non-causal; c >= 1: block-causal with block c (1 = ordinary causal). */
+  int64_t causal_block_size;
+  /* P, the number of virtual ring ranks; 1 <= P <= 64 and S % P == 0. */
+  int64_t ring_size;
+  /* If use_ring_order != 0, step t visits key/value block
+   * (r - ring_order[t]) mod P instead of (r - t) mod P; ring_order must be a
+   * permutation of 0..P-1 (RA_ERR_ORDER otherwise). */
+  int32_t ring_order[RA_MAX_RING];
+  int32_t use_ring_order;
+  int32_t reserved;   /* must be 0 */
+} ra_params;
+
+/* Workspace bytes (device memory, caller-allocated, 256-byte aligned base)
+ * needed by ra_forward (which = 0) or ra_backward (which = 1) for a problem
+ * shaped like q.  has_bias / has_segments say whether attention_bias /
+ * segment_ids will be passed.  Returns 0 when none is needed, or
+ * (size_t)-1 for invalid arguments. */
+size_t ra_workspace_size(int which, const ra_tensor* q, const ra_params* p, int has_bias, int has_segments);
+
+/* Forward: o = softmax(q k^T / sqrt(D) + bias, masked) v and its
+ * log-sum-exp, every query tile visiting the key/value tiles in ring order
+ * ("Ring Attention技术解析" §2.2) with the exact online-softmax merge.
+ *  q, k, v: [B,S,H,D], all bf16 (sm_100a tensor-core path) or all fp32
+ *           (CUDA-core fp32 path).
+ *  attention_bias, segment_ids: may be NULL (see conventions).
+ *  o: [B,S,H,D], dtype of q (bf16 rounded to nearest even).  lse: fp32 [B,H,S].
+ *  workspace: device buffer of at least ra_workspace_size(0, ...) bytes
+ *  (may be NULL when that size is 0).  Contents are scratch. */
+int ra_forward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* attention_bias,
+               const ra_tensor* segment_ids, const ra_params* p, ra_tensor* o, ra_tensor* lse, void* workspace,
+               size_t workspace_bytes, void* stream);
+
+/* Backward of ra_forward given the upstream gradient dO, recomputing the
+ * attention probabilities from q, k and the saved lse (the recompute policy
+ * "nothing_saveable" of "RingAttention核心功能全解析" 核心API调用):
+ *   Delta_i = <dO_i, o_i>, P_ij = exp(s_ij - lse_i), dP_ij = <dO_i, v_j>,
+ *   dS_ij = P_ij (dP_ij - Delta_i), dq = dS k / sqrt(D), dk = dS^T q / sqrt(D),
+ *   dv = P^T dO.
+ *  q, k, v, o, d_o: same dtype (bf16 or fp32), [B,S,H,D]; lse fp32 [B,H,S]
+ *  as written by ra_forward.  dq, dk, dv: [B,S,H,D] (bf16 or fp32; with
+ *  fp32 inputs they must be fp32).  workspace: at least
+ *  ra_workspace_size(1, ...) bytes (holds Delta and an fp32 dq accumulator). */
+int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* o,
+                const ra_tensor* d_o, const ra_tensor* lse, const ra_tensor* attention_bias,
+                const ra_tensor* segment_ids, const ra_params* p, ra_tensor* dq, ra_tensor* dk, ra_tensor* dv,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* One ring step ("Ring Attention技术解析" §2.2, one iteration of the loop):
+ * the local query block q_blk [B,Sq,H,D] (tokens q_off .. q_off+Sq-1 of the
+ * sequence) attends to one visiting key/value block k_blk, v_blk [B,Sk,H,D]
+ * (tokens k_off ..), updating the caller-held running state in place:
+ *   o_acc fp32 [B,Sq,H,D] (unnormalised output), m, l fp32 [B,H,Sq]
+ *   (running max in natural-log units, running sum).
+ * Initialise m = -inf, l = 0, o_acc = 0 before the first step; any step
+ * order gives the same finalized result.  bias_blk: NULL or fp32 [B,Sk] for
+ * the visiting keys; seg_q / seg_k: both NULL or int32 [B,Sq] / [B,Sk].
+ * Only p->causal_block_size is used from p.  q/k/v bf16 or fp32 (fp32
+ * arithmetic, CUDA cores). */
+int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_blk, int64_t q_off, int64_t k_off,
+            const ra_tensor* bias_blk, const ra_tensor* seg_q, const ra_tensor* seg_k, const ra_params* p,
+            ra_tensor* o_acc, ra_tensor* m, ra_tensor* l, void* stream);
+
+/* Finalize a running state: o = o_acc / l (bf16 or fp32 output), lse = m +
+ * log(l); rows with l == 0 give o = 0 and lse = -inf. */
+int ra_finalize(const ra_tensor* o_acc, const ra_tensor* m, const ra_tensor* l, ra_tensor* o, ra_tensor* lse,
+                void* stream);
+
+/* Merge two normalised partial results computed over disjoint key sets:
+ *   lse = max(a,b) + log1p(exp(-|lse_a - lse_b|)),
+ *   o   = o_a exp(lse_a - lse) + o_b exp(lse_b - lse).
+ * o_* [B,S,H,D] (all bf16 or all fp32), lse_* fp32 [B,H,S].  o_out / lse_out
+ * may alias o_a / lse_a (element-wise in place). */
+int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* o_b, const ra_tensor* lse_b,
+                 ra_tensor* o_out, ra_tensor* lse_out, void* stream);
+
+/* Synchronizes `stream`, returns the device status word of the current
+ * device (RA_OK or RA_ERR_DEVICE_TIMEOUT) and clears it.  RA_ERR_CUDA if
+ * the synchronization itself failed. */
+int ra_get_device_status(void* stream);
+
+/* Static description of an error code (never NULL). */
+const char* ra_strerror(int code);
+
+/* Host-only introspection (no device work).
+ * Exact number of visible (query, key) pairs summed over batch and heads,
+ * from the same mask rules the kernels use.  seg_host: NULL or int32 [B*S]
+ * row-major (host memory); bias_host: NULL or fp32 [B*S] (host).  Returns
+ * -1 on invalid arguments. */
+int64_t ra_count_visible_pairs(int64_t B, int64_t S, int64_t H, int64_t causal_block_size,
+                               const int32_t* seg_host, const float* bias_host);
+
+/* Host-only introspection: the key/value tile indices (128-token tiles),
+ * in visiting order, that the query rows [q_first, q_last] of batch row 0
+ * visit on the ring: step t covers the tiles of block (r - order[t]) mod P,
+ * r = q_first's ring block; tiles that masking hides from every row of the
+ * range are skipped.  seg_host / bias_host as in ra_count_visible_pairs
+ * (batch row 0 only).  Writes at most `cap` indices to out_host and returns
+ * the full count, or -1 on invalid arguments. */
+int64_t ra_ring_schedule(int64_t S, const ra_params* p, int64_t q_first, int64_t q_last, const int32_t* seg_host,
+                         const float* bias_host, int32_t* out_host, int64_t cap);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RINGATTN_H_ */

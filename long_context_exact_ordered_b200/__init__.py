@@ -1,0 +1,26 @@
+"""B200-native Ring Attention: blockwise exact attention over virtual ring ranks.
+
+The compute path is ``libringattn.so`` (hand-written sm_100a CUDA behind a C
+ABI, include/ringattn.h); this package only marshals torch tensors into it.
+"""
+
+from .api import (  # noqa: F401
+    RingAttentionFunction,
+    count_visible_pairs,
+    device_status,
+    finalize,
+    init_state,
+    lse_merge,
+    ring_schedule,
+    ring_step,
+    ringattention,
+    ringattention_backward,
+    workspace_size,
+)
+from ._lib import RingAttnError, load  # noqa: F401
+
+__all__ = [
+    "ringattention", "ringattention_backward", "ring_step", "init_state", "finalize", "lse_merge",
+    "device_status", "count_visible_pairs", "ring_schedule", "workspace_size", "RingAttentionFunction",
+    "RingAttnError", "load",
+]

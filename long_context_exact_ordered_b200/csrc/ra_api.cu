@@ -1,0 +1,641 @@
+// C ABI of the library (declared in include/ringattn.h): argument checks,
+// workspace layout, TMA tensor maps, kernel launches, and the host-only
+// schedule / visible-pair introspection.  Single translation unit: every
+// kernel header is included here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/ringattn.h"
+#include "ra_common.cuh"
+#include "ra_fwd_sm100.cuh"
+#include "ra_bwd_sm100.cuh"
+#include "ra_simt.cuh"
+
+using namespace ra;
+
+namespace {
+
+// ---------------------------------------------------------------- validation
+
+bool is_dtype(const ra_tensor* t, int dt) { return t && t->dtype == dt; }
+
+// [B, S, H, D] with contiguous last dim.
+int check_bshd(const ra_tensor* t, int64_t B, int64_t S, int64_t H, int64_t D) {
+  if (!t) return RA_ERR_NULL;
+  if (t->ndim != 4) return RA_ERR_SHAPE;
+  if (t->shape[0] != B || t->shape[1] != S || t->shape[2] != H || t->shape[3] != D) return RA_ERR_SHAPE;
+  if (t->stride[3] != 1) return RA_ERR_STRIDE;
+  if (!t->data && B * S * H * D > 0) return RA_ERR_NULL;
+  return RA_OK;
+}
+
+// bf16 operand read by TMA / written with 16-byte vector stores.
+int check_tma_bf16(const ra_tensor* t) {
+  if (reinterpret_cast<uintptr_t>(t->data) % 16) return RA_ERR_STRIDE;
+  for (int i = 0; i < 3; ++i) {
+    if ((t->stride[i] * 2) % 16) return RA_ERR_STRIDE;
+    if (t->stride[i] < 0 || t->stride[i] * 2 >= (int64_t(1) << 40)) return RA_ERR_STRIDE;
+  }
+  return RA_OK;
+}
+
+// [B, H, S] fp32 (lse, m, l).
+int check_bhs(const ra_tensor* t, int64_t B, int64_t H, int64_t S) {
+  if (!t) return RA_ERR_NULL;
+  if (t->ndim != 3) return RA_ERR_SHAPE;
+  if (t->shape[0] != B || t->shape[1] != H || t->shape[2] != S) return RA_ERR_SHAPE;
+  if (t->dtype != RA_F32) return RA_ERR_DTYPE;
+  if (!t->data && B * H * S > 0) return RA_ERR_NULL;
+  return RA_OK;
+}
+
+// [B, S] (bias fp32 / segment ids int32), optional.
+int check_bs(const ra_tensor* t, int64_t B, int64_t S, int dtype) {
+  if (!t) return RA_OK;
+  if (t->ndim != 2) return RA_ERR_SHAPE;
+  if (t->shape[0] != B || t->shape[1] != S) return RA_ERR_SHAPE;
+  if (t->dtype != dtype) return RA_ERR_DTYPE;
+  if (!t->data && B * S > 0) return RA_ERR_NULL;
+  return RA_OK;
+}
+
+#define RA_TRY(x)               \
+  do {                          \
+    int _e = (x);               \
+    if (_e != RA_OK) return _e; \
+  } while (0)
+
+int make_ring(const ra_params* p, int64_t S, RingDesc* rd) {
+  if (!p) return RA_ERR_NULL;
+  if (p->reserved != 0) return RA_ERR_UNSUPPORTED;
+  if (p->ring_size < 1) return RA_ERR_DIVISIBILITY;
+  if (p->ring_size > kMaxRing) return RA_ERR_UNSUPPORTED;
+  if (p->causal_block_size < 0) return RA_ERR_DIVISIBILITY;
+  if (S % p->ring_size) return RA_ERR_DIVISIBILITY;
+  const int64_t blk = S / p->ring_size;
+  if (p->query_chunk_size < 1 || p->key_chunk_size < 1) return RA_ERR_DIVISIBILITY;
+  if (blk > 0 && (blk % p->query_chunk_size || blk % p->key_chunk_size)) return RA_ERR_DIVISIBILITY;
+  if (p->causal_block_size > INT32_MAX || S > (int64_t(1) << 31) - kTile) return RA_ERR_UNSUPPORTED;
+  std::memset(rd, 0, sizeof(*rd));
+  rd->S = S;
+  rd->blk = blk > 0 ? blk : 1;
+  rd->P = (int32_t)p->ring_size;
+  rd->ntiles = (int32_t)ceil_div64(S, kTile);
+  rd->cbs = (int32_t)p->causal_block_size;
+  bool seen[kMaxRing] = {false};
+  for (int t = 0; t < rd->P; ++t) {
+    int32_t o = p->use_ring_order ? p->ring_order[t] : t;
+    if (o < 0 || o >= rd->P || seen[o]) return RA_ERR_ORDER;
+    seen[o] = true;
+    rd->order[t] = o;
+  }
+  return RA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct WsLayout {
+  size_t meta = 0, delta = 0, dqacc = 0, total = 0;
+};
+
+WsLayout ws_layout(int which, int64_t B, int64_t S, int64_t H, int64_t D, bool need_meta) {
+  WsLayout w;
+  size_t off = 0;
+  if (need_meta) {
+    w.meta = off;
+    off += align256((size_t)B * ceil_div64(S, kTile) * sizeof(int4));
+  }
+  if (which == 1) {
+    w.delta = off;
+    off += align256((size_t)B * H * S * sizeof(float));
+    w.dqacc = off;
+    off += align256((size_t)B * H * S * D * sizeof(float));
+  }
+  w.total = off;
+  return w;
+}
+
+// ---------------------------------------------------------------- device facts
+
+int device_cc_major() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return -1;
+  return major;
+}
+
+// ---------------------------------------------------------------- TMA maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// bf16 [B, S, H, D] -> 4-D map (D, H, S, B), box 64 x 1 x rows x 1, 128-byte swizzle.
+int make_tmap_bshd(CUtensorMap* m, const ra_tensor* t, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return RA_ERR_CUDA;
+  cuuint64_t dims[4] = {(cuuint64_t)t->shape[3], (cuuint64_t)t->shape[2], (cuuint64_t)t->shape[1],
+                        (cuuint64_t)t->shape[0]};
+  cuuint64_t strides[3] = {(cuuint64_t)t->stride[2] * 2, (cuuint64_t)t->stride[1] * 2, (cuuint64_t)t->stride[0] * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RA_OK : RA_ERR_CUDA;
+}
+
+int last_cuda() { return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA; }
+
+MaskArgs mask_args(const ra_tensor* bias, const ra_tensor* seg) {
+  MaskArgs mk{};
+  if (seg) {
+    mk.seg = static_cast<const int32_t*>(seg->data);
+    mk.seg_sb = seg->stride[0];
+    mk.seg_ss = seg->stride[1];
+  }
+  if (bias) {
+    mk.bias = static_cast<const float*>(bias->data);
+    mk.bias_sb = bias->stride[0];
+    mk.bias_ss = bias->stride[1];
+  }
+  return mk;
+}
+
+int launch_meta(const MaskArgs& mk, int64_t B, const RingDesc& rd, int4* meta, cudaStream_t st) {
+  dim3 grid(rd.ntiles, (unsigned)B);
+  tile_meta_kernel<<<grid, 128, 0, st>>>(mk, rd.S, rd.ntiles, meta);
+  return last_cuda();
+}
+
+template <int D>
+int launch_fwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const MaskArgs& mk,
+                     const RingDesc& rd, const int4* meta, ra_tensor* o, ra_tensor* lse, cudaStream_t st) {
+  using L = FwdLayout<D>;
+  CUtensorMap tq, tk, tv;
+  RA_TRY(make_tmap_bshd(&tq, q, kTile));
+  RA_TRY(make_tmap_bshd(&tk, k, kTile));
+  RA_TRY(make_tmap_bshd(&tv, v, kTile));
+  FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.rd = rd;
+  prm.B = (int32_t)q->shape[0];
+  prm.H = (int32_t)q->shape[2];
+  prm.npairs = (rd.ntiles + 1) / 2;
+  prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  prm.o = static_cast<__nv_bfloat16*>(o->data);
+  prm.o_sb = o->stride[0];
+  prm.o_ss = o->stride[1];
+  prm.o_sh = o->stride[2];
+  prm.lse = static_cast<float*>(lse->data);
+  prm.lse_sb = lse->stride[0];
+  prm.lse_sh = lse->stride[1];
+  prm.lse_ss = lse->stride[2];
+  prm.seg = mk.seg;
+  prm.seg_sb = mk.seg_sb;
+  prm.seg_ss = mk.seg_ss;
+  prm.bias = mk.bias;
+  prm.bias_sb = mk.bias_sb;
+  prm.bias_ss = mk.bias_ss;
+  prm.meta = meta;
+  const int64_t grid = (int64_t)prm.npairs * prm.B * prm.H;
+  if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(ra_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
+      cudaSuccess)
+    return RA_ERR_CUDA;
+  {
+    // The register split must fit in what the block is launched with.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, ra_fwd_sm100_kernel<D>) != cudaSuccess) return RA_ERR_CUDA;
+    if (128 * L::REGS_LOW + 256 * L::REGS_HIGH > L::THREADS * fa.numRegs) return RA_ERR_UNSUPPORTED;
+  }
+  ra_fwd_sm100_kernel<D><<<(unsigned)grid, 384, L::SMEM_ALLOC, st>>>(tq, tk, tv, prm);
+  return last_cuda();
+}
+
+View4 view4(const ra_tensor* t) { return View4{t->data, t->stride[0], t->stride[1], t->stride[2]}; }
+OutView4 oview4(ra_tensor* t) { return OutView4{t->data, t->stride[0], t->stride[1], t->stride[2]}; }
+
+template <int D, typename T>
+int launch_fwd_simt(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const MaskArgs& mk,
+                    const RingDesc& rd, const int4* meta, ra_tensor* o, ra_tensor* lse, cudaStream_t st) {
+  SimtFwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.rd = rd;
+  a.B = (int)q->shape[0];
+  a.H = (int)q->shape[2];
+  a.scale = (float)(1.0 / std::sqrt((double)D));
+  a.mk = mk;
+  a.meta = meta;
+  a.q = view4(q);
+  a.k = view4(k);
+  a.v = view4(v);
+  a.o = oview4(o);
+  a.lse = static_cast<float*>(lse->data);
+  a.lse_sb = lse->stride[0];
+  a.lse_sh = lse->stride[1];
+  a.lse_ss = lse->stride[2];
+  const int smem = SimtSmem<D>::BYTES;
+  if (cudaFuncSetAttribute(simt_fwd_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return RA_ERR_CUDA;
+  dim3 grid((unsigned)ceil_div64(rd.S, kSimtRows), (unsigned)(a.B * a.H));
+  simt_fwd_kernel<D, T><<<grid, kSimtRows, smem, st>>>(a);
+  return last_cuda();
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+
+extern "C" {
+
+const char* ra_strerror(int code) {
+  switch (code) {
+    case RA_OK: return "ok";
+    case RA_ERR_NULL: return "a required pointer is NULL";
+    case RA_ERR_DTYPE: return "unsupported or mismatched dtype";
+    case RA_ERR_SHAPE: return "rank or shape mismatch";
+    case RA_ERR_STRIDE: return "head dim not contiguous or TMA alignment violated (16-byte base and strides)";
+    case RA_ERR_DIVISIBILITY: return "S must be divisible by ring_size, and S/ring_size by both chunk sizes";
+    case RA_ERR_UNSUPPORTED: return "unsupported configuration (head_dim, ring_size, device or size limits)";
+    case RA_ERR_WORKSPACE: return "workspace missing or too small";
+    case RA_ERR_CUDA: return "CUDA runtime error";
+    case RA_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait ran out";
+    case RA_ERR_ORDER: return "ring_order is not a permutation of 0..ring_size-1";
+    default: return "unknown error";
+  }
+}
+
+size_t ra_workspace_size(int which, const ra_tensor* q, const ra_params* p, int has_bias, int has_segments) {
+  if (!q || !p || q->ndim != 4 || (which != 0 && which != 1)) return (size_t)-1;
+  return ws_layout(which, q->shape[0], q->shape[1], q->shape[2], q->shape[3], has_bias || has_segments).total;
+}
+
+int ra_forward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* attention_bias,
+               const ra_tensor* segment_ids, const ra_params* p, ra_tensor* o, ra_tensor* lse, void* workspace,
+               size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !p) return RA_ERR_NULL;
+  if (q->ndim != 4) return RA_ERR_SHAPE;
+  const int64_t B = q->shape[0], S = q->shape[1], H = q->shape[2], D = q->shape[3];
+  if (B < 0 || S < 0 || H < 0) return RA_ERR_SHAPE;
+  RA_TRY(check_bshd(q, B, S, H, D));
+  RA_TRY(check_bshd(k, B, S, H, D));
+  RA_TRY(check_bshd(v, B, S, H, D));
+  RA_TRY(check_bshd(o, B, S, H, D));
+  RA_TRY(check_bhs(lse, B, H, S));
+  RA_TRY(check_bs(attention_bias, B, S, RA_F32));
+  RA_TRY(check_bs(segment_ids, B, S, RA_I32));
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const int dt = q->dtype;
+  if (dt != RA_BF16 && dt != RA_F32) return RA_ERR_DTYPE;
+  if (!is_dtype(k, dt) || !is_dtype(v, dt) || !is_dtype(o, dt)) return RA_ERR_DTYPE;
+  if (B * S * H == 0) {
+    RingDesc rd;
+    return make_ring(p, S, &rd) == RA_ERR_ORDER ? RA_ERR_ORDER : RA_OK;
+  }
+  RingDesc rd;
+  RA_TRY(make_ring(p, S, &rd));
+  if (dt == RA_BF16) {
+    RA_TRY(check_tma_bf16(q));
+    RA_TRY(check_tma_bf16(k));
+    RA_TRY(check_tma_bf16(v));
+    RA_TRY(check_tma_bf16(o));
+  }
+  const bool need_meta = attention_bias || segment_ids;
+  const WsLayout w = ws_layout(0, B, S, H, D, need_meta);
+  if (w.total > 0 && (!workspace || workspace_bytes < w.total)) return RA_ERR_WORKSPACE;
+  if (w.total > 0 && reinterpret_cast<uintptr_t>(workspace) % 256) return RA_ERR_WORKSPACE;
+  if (dt == RA_BF16) {
+    const int major = device_cc_major();
+    if (major < 0) return RA_ERR_CUDA;
+    if (major != 10) return RA_ERR_UNSUPPORTED;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const MaskArgs mk = mask_args(attention_bias, segment_ids);
+  int4* meta = need_meta ? reinterpret_cast<int4*>(static_cast<char*>(workspace) + w.meta) : nullptr;
+  if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
+  if (dt == RA_BF16) {
+    return D == 64 ? launch_fwd_sm100<64>(q, k, v, mk, rd, meta, o, lse, st)
+                   : launch_fwd_sm100<128>(q, k, v, mk, rd, meta, o, lse, st);
+  }
+  return D == 64 ? launch_fwd_simt<64, float>(q, k, v, mk, rd, meta, o, lse, st)
+                 : launch_fwd_simt<128, float>(q, k, v, mk, rd, meta, o, lse, st);
+}
+
+int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* o,
+                const ra_tensor* d_o, const ra_tensor* lse, const ra_tensor* attention_bias,
+                const ra_tensor* segment_ids, const ra_params* p, ra_tensor* dq, ra_tensor* dk, ra_tensor* dv,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !d_o || !lse || !p || !dq || !dk || !dv) return RA_ERR_NULL;
+  if (q->ndim != 4) return RA_ERR_SHAPE;
+  const int64_t B = q->shape[0], S = q->shape[1], H = q->shape[2], D = q->shape[3];
+  if (B < 0 || S < 0 || H < 0) return RA_ERR_SHAPE;
+  for (const ra_tensor* t : {q, k, v, o, d_o, (const ra_tensor*)dq, (const ra_tensor*)dk, (const ra_tensor*)dv})
+    RA_TRY(check_bshd(t, B, S, H, D));
+  RA_TRY(check_bhs(lse, B, H, S));
+  RA_TRY(check_bs(attention_bias, B, S, RA_F32));
+  RA_TRY(check_bs(segment_ids, B, S, RA_I32));
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const int dt = q->dtype;
+  if (dt != RA_BF16 && dt != RA_F32) return RA_ERR_DTYPE;
+  for (const ra_tensor* t : {k, v, o, d_o})
+    if (!is_dtype(t, dt)) return RA_ERR_DTYPE;
+  for (const ra_tensor* t : {(const ra_tensor*)dq, (const ra_tensor*)dk, (const ra_tensor*)dv}) {
+    if (t->dtype != RA_BF16 && t->dtype != RA_F32) return RA_ERR_DTYPE;
+    if (dt == RA_F32 && t->dtype != RA_F32) return RA_ERR_DTYPE;
+  }
+  RingDesc rd;
+  if (B * S * H == 0) return make_ring(p, S, &rd) == RA_ERR_ORDER ? RA_ERR_ORDER : RA_OK;
+  RA_TRY(make_ring(p, S, &rd));
+  if (dt == RA_BF16)
+    for (const ra_tensor* t : {q, k, v, o, d_o}) RA_TRY(check_tma_bf16(t));
+  const bool need_meta = attention_bias || segment_ids;
+  const WsLayout w = ws_layout(1, B, S, H, D, need_meta);
+  if (!workspace || workspace_bytes < w.total || reinterpret_cast<uintptr_t>(workspace) % 256)
+    return RA_ERR_WORKSPACE;
+  if (dt == RA_BF16) {
+    const int major = device_cc_major();
+    if (major < 0) return RA_ERR_CUDA;
+    if (major != 10) return RA_ERR_UNSUPPORTED;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const MaskArgs mk = mask_args(attention_bias, segment_ids);
+  char* ws = static_cast<char*>(workspace);
+  int4* meta = need_meta ? reinterpret_cast<int4*>(ws + w.meta) : nullptr;
+  float* delta = reinterpret_cast<float*>(ws + w.delta);
+  float* dqacc = reinterpret_cast<float*>(ws + w.dqacc);
+  if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
+  {
+    BwdPreArgs pa{(int)B, (int)S, (int)H, (int)D, o->data, o->stride[0], o->stride[1], o->stride[2],
+                  d_o->data, d_o->stride[0], d_o->stride[1], d_o->stride[2], dt == RA_BF16, delta};
+    const int64_t threads = B * S * H * 32;
+    bwd_pre_kernel<<<(unsigned)ceil_div64(threads, 256), 256, 0, st>>>(pa);
+    RA_TRY(last_cuda());
+  }
+  if (dt == RA_BF16) {
+    return D == 64 ? launch_bwd_sm100<64>(q, k, v, d_o, lse, mk, rd, meta, delta, dqacc, dq, dk, dv, st)
+                   : launch_bwd_sm100<128>(q, k, v, d_o, lse, mk, rd, meta, delta, dqacc, dq, dk, dv, st);
+  }
+  SimtBwdArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.rd = rd;
+  a.B = (int)B;
+  a.H = (int)H;
+  a.scale = (float)(1.0 / std::sqrt((double)D));
+  a.mk = mk;
+  a.q = view4(q);
+  a.k = view4(k);
+  a.v = view4(v);
+  a.dO = view4(d_o);
+  a.lse = static_cast<const float*>(lse->data);
+  a.lse_sb = lse->stride[0];
+  a.lse_sh = lse->stride[1];
+  a.lse_ss = lse->stride[2];
+  a.delta = delta;
+  a.dq = oview4(dq);
+  a.dk = oview4(dk);
+  a.dv = oview4(dv);
+  dim3 grid((unsigned)ceil_div64(S, 64), (unsigned)(B * H));
+  if (D == 64) {
+    simt_bwd_dq_kernel<64><<<grid, 64, 0, st>>>(a);
+    simt_bwd_dkdv_kernel<64><<<grid, 64, 0, st>>>(a);
+  } else {
+    simt_bwd_dq_kernel<128><<<grid, 64, 0, st>>>(a);
+    simt_bwd_dkdv_kernel<128><<<grid, 64, 0, st>>>(a);
+  }
+  return last_cuda();
+}
+
+int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_blk, int64_t q_off, int64_t k_off,
+            const ra_tensor* bias_blk, const ra_tensor* seg_q, const ra_tensor* seg_k, const ra_params* p,
+            ra_tensor* o_acc, ra_tensor* m, ra_tensor* l, void* stream) {
+  if (!q_blk || !k_blk || !v_blk || !p || !o_acc || !m || !l) return RA_ERR_NULL;
+  if (q_blk->ndim != 4 || k_blk->ndim != 4) return RA_ERR_SHAPE;
+  const int64_t B = q_blk->shape[0], Sq = q_blk->shape[1], H = q_blk->shape[2], D = q_blk->shape[3];
+  const int64_t Sk = k_blk->shape[1];
+  if (B < 0 || Sq < 0 || Sk < 0 || H < 0) return RA_ERR_SHAPE;
+  RA_TRY(check_bshd(q_blk, B, Sq, H, D));
+  RA_TRY(check_bshd(k_blk, B, Sk, H, D));
+  RA_TRY(check_bshd(v_blk, B, Sk, H, D));
+  RA_TRY(check_bshd(o_acc, B, Sq, H, D));
+  RA_TRY(check_bhs(m, B, H, Sq));
+  RA_TRY(check_bhs(l, B, H, Sq));
+  RA_TRY(check_bs(bias_blk, B, Sk, RA_F32));
+  if ((seg_q == nullptr) != (seg_k == nullptr)) return RA_ERR_NULL;
+  RA_TRY(check_bs(seg_q, B, Sq, RA_I32));
+  RA_TRY(check_bs(seg_k, B, Sk, RA_I32));
+  if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
+  const int dt = q_blk->dtype;
+  if (dt != RA_BF16 && dt != RA_F32) return RA_ERR_DTYPE;
+  if (!is_dtype(k_blk, dt) || !is_dtype(v_blk, dt) || o_acc->dtype != RA_F32) return RA_ERR_DTYPE;
+  if (p->causal_block_size < 0 || q_off < 0 || k_off < 0) return RA_ERR_DIVISIBILITY;
+  if (B * Sq * H == 0 || Sk == 0) return RA_OK;
+  SimtStepArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.B = (int)B;
+  a.H = (int)H;
+  a.D = (int)D;
+  a.Sq = Sq;
+  a.Sk = Sk;
+  a.q_off = q_off;
+  a.k_off = k_off;
+  a.cbs = (int32_t)p->causal_block_size;
+  a.scale = (float)(1.0 / std::sqrt((double)D));
+  a.q = view4(q_blk);
+  a.k = view4(k_blk);
+  a.v = view4(v_blk);
+  if (seg_q) {
+    a.seg_q = static_cast<const int32_t*>(seg_q->data);
+    a.segq_sb = seg_q->stride[0];
+    a.segq_ss = seg_q->stride[1];
+    a.seg_k = static_cast<const int32_t*>(seg_k->data);
+    a.segk_sb = seg_k->stride[0];
+    a.segk_ss = seg_k->stride[1];
+  }
+  if (bias_blk) {
+    a.bias = static_cast<const float*>(bias_blk->data);
+    a.bias_sb = bias_blk->stride[0];
+    a.bias_ss = bias_blk->stride[1];
+  }
+  a.acc = static_cast<float*>(o_acc->data);
+  a.acc_sb = o_acc->stride[0];
+  a.acc_ss = o_acc->stride[1];
+  a.acc_sh = o_acc->stride[2];
+  a.m = static_cast<float*>(m->data);
+  a.l = static_cast<float*>(l->data);
+  if (m->stride[0] != l->stride[0] || m->stride[1] != l->stride[1] || m->stride[2] != l->stride[2])
+    return RA_ERR_STRIDE;
+  a.ml_sb = m->stride[0];
+  a.ml_sh = m->stride[1];
+  a.ml_ss = m->stride[2];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid((unsigned)ceil_div64(Sq, kSimtRows), (unsigned)(B * H));
+  if (D == 64) {
+    const int smem = SimtSmem<64>::BYTES;
+    if (dt == RA_BF16) {
+      if (cudaFuncSetAttribute(simt_step_kernel<64, __nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem) != cudaSuccess)
+        return RA_ERR_CUDA;
+      simt_step_kernel<64, __nv_bfloat16><<<grid, kSimtRows, smem, st>>>(a);
+    } else {
+      if (cudaFuncSetAttribute(simt_step_kernel<64, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return RA_ERR_CUDA;
+      simt_step_kernel<64, float><<<grid, kSimtRows, smem, st>>>(a);
+    }
+  } else {
+    const int smem = SimtSmem<128>::BYTES;
+    if (dt == RA_BF16) {
+      if (cudaFuncSetAttribute(simt_step_kernel<128, __nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               smem) != cudaSuccess)
+        return RA_ERR_CUDA;
+      simt_step_kernel<128, __nv_bfloat16><<<grid, kSimtRows, smem, st>>>(a);
+    } else {
+      if (cudaFuncSetAttribute(simt_step_kernel<128, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess)
+        return RA_ERR_CUDA;
+      simt_step_kernel<128, float><<<grid, kSimtRows, smem, st>>>(a);
+    }
+  }
+  return last_cuda();
+}
+
+int ra_finalize(const ra_tensor* o_acc, const ra_tensor* m, const ra_tensor* l, ra_tensor* o, ra_tensor* lse,
+                void* stream) {
+  if (!o_acc || !m || !l || !o || !lse) return RA_ERR_NULL;
+  if (o_acc->ndim != 4) return RA_ERR_SHAPE;
+  const int64_t B = o_acc->shape[0], S = o_acc->shape[1], H = o_acc->shape[2], D = o_acc->shape[3];
+  RA_TRY(check_bshd(o_acc, B, S, H, D));
+  RA_TRY(check_bshd(o, B, S, H, D));
+  RA_TRY(check_bhs(m, B, H, S));
+  RA_TRY(check_bhs(l, B, H, S));
+  RA_TRY(check_bhs(lse, B, H, S));
+  if (o_acc->dtype != RA_F32) return RA_ERR_DTYPE;
+  if (o->dtype != RA_F32 && o->dtype != RA_BF16) return RA_ERR_DTYPE;
+  if (m->stride[0] != l->stride[0] || m->stride[1] != l->stride[1] || m->stride[2] != l->stride[2])
+    return RA_ERR_STRIDE;
+  const int64_t n = B * S * H;
+  if (n == 0) return RA_OK;
+  FinalizeArgs a{(int)B, (int)S, (int)H, (int)D,
+                 static_cast<const float*>(o_acc->data), o_acc->stride[0], o_acc->stride[1], o_acc->stride[2],
+                 static_cast<const float*>(m->data), static_cast<const float*>(l->data),
+                 m->stride[0], m->stride[1], m->stride[2],
+                 o->data, o->stride[0], o->stride[1], o->stride[2], o->dtype == RA_BF16,
+                 static_cast<float*>(lse->data), lse->stride[0], lse->stride[1], lse->stride[2]};
+  finalize_kernel<<<(unsigned)ceil_div64(n, 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return last_cuda();
+}
+
+int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* o_b, const ra_tensor* lse_b,
+                 ra_tensor* o_out, ra_tensor* lse_out, void* stream) {
+  if (!o_a || !lse_a || !o_b || !lse_b || !o_out || !lse_out) return RA_ERR_NULL;
+  if (o_a->ndim != 4) return RA_ERR_SHAPE;
+  const int64_t B = o_a->shape[0], S = o_a->shape[1], H = o_a->shape[2], D = o_a->shape[3];
+  RA_TRY(check_bshd(o_a, B, S, H, D));
+  RA_TRY(check_bshd(o_b, B, S, H, D));
+  RA_TRY(check_bshd(o_out, B, S, H, D));
+  RA_TRY(check_bhs(lse_a, B, H, S));
+  RA_TRY(check_bhs(lse_b, B, H, S));
+  RA_TRY(check_bhs(lse_out, B, H, S));
+  const int dt = o_a->dtype;
+  if (dt != RA_F32 && dt != RA_BF16) return RA_ERR_DTYPE;
+  if (o_b->dtype != dt || o_out->dtype != dt) return RA_ERR_DTYPE;
+  const int64_t n = B * S * H;
+  if (n == 0) return RA_OK;
+  MergeArgs a{(int)B, (int)S, (int)H, (int)D,
+              o_a->data, o_a->stride[0], o_a->stride[1], o_a->stride[2],
+              static_cast<const float*>(lse_a->data), lse_a->stride[0], lse_a->stride[1], lse_a->stride[2],
+              o_b->data, o_b->stride[0], o_b->stride[1], o_b->stride[2],
+              static_cast<const float*>(lse_b->data), lse_b->stride[0], lse_b->stride[1], lse_b->stride[2],
+              o_out->data, o_out->stride[0], o_out->stride[1], o_out->stride[2],
+              static_cast<float*>(lse_out->data), lse_out->stride[0], lse_out->stride[1], lse_out->stride[2],
+              dt == RA_BF16};
+  lse_merge_kernel<<<(unsigned)ceil_div64(n, 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return last_cuda();
+}
+
+int ra_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, ra::g_ra_status, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(ra::g_ra_status, &zero, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  return v;
+}
+
+int64_t ra_count_visible_pairs(int64_t B, int64_t S, int64_t H, int64_t causal_block_size, const int32_t* seg_host,
+                               const float* bias_host) {
+  if (B < 0 || S < 0 || H < 0 || causal_block_size < 0) return -1;
+  int64_t total = 0;
+  for (int64_t b = 0; b < B; ++b) {
+    const int32_t* sg = seg_host ? seg_host + b * S : nullptr;
+    const float* bs = bias_host ? bias_host + b * S : nullptr;
+    std::unordered_map<int32_t, int64_t> cnt;   // visible-key count per segment id so far
+    auto key_ok = [&](int64_t j) { return !bs || bs[j] > -INFINITY; };
+    const int64_t c = causal_block_size > 0 ? causal_block_size : S;
+    for (int64_t a = 0; a < S; a += c) {
+      const int64_t e = a + c < S ? a + c : S;
+      for (int64_t j = a; j < e; ++j)        // keys of this causal block become visible
+        if (key_ok(j)) ++cnt[sg ? sg[j] : 0];
+      for (int64_t i = a; i < e; ++i) {      // queries of the block see every key so far
+        auto f = cnt.find(sg ? sg[i] : 0);
+        if (f != cnt.end()) total += f->second;
+      }
+    }
+  }
+  return total * H;
+}
+
+int64_t ra_ring_schedule(int64_t S, const ra_params* p, int64_t q_first, int64_t q_last, const int32_t* seg_host,
+                         const float* bias_host, int32_t* out_host, int64_t cap) {
+  RingDesc rd;
+  if (S < 1 || make_ring(p, S, &rd) != RA_OK) return -1;
+  if (q_first < 0 || q_last < q_first || q_first >= S) return -1;
+  std::vector<int4> meta;
+  if (seg_host || bias_host) {
+    meta.resize(rd.ntiles);
+    for (int32_t t = 0; t < rd.ntiles; ++t) {
+      int smin = INT32_MAX, smax = INT32_MIN, any = 0, zero = 1;
+      for (int64_t j = (int64_t)t * kTile; j < S && j < (int64_t)(t + 1) * kTile; ++j) {
+        const int s = seg_host ? seg_host[j] : 0;
+        smin = s < smin ? s : smin;
+        smax = s > smax ? s : smax;
+        if (bias_host) {
+          any |= bias_host[j] > -INFINITY;
+          zero &= bias_host[j] == 0.0f;
+        } else {
+          any = 1;
+        }
+      }
+      meta[t] = make_int4(smin, smax, (any ? kMetaAnyFinite : 0) | (zero ? kMetaAllZero : 0), 0);
+    }
+  }
+  KvIter it;
+  kv_iter_init(it, rd, q_first, q_last, meta.empty() ? nullptr : meta.data(), seg_host != nullptr,
+               bias_host != nullptr);
+  int64_t n = 0;
+  for (int32_t t = kv_iter_next(it, rd); t >= 0; t = kv_iter_next(it, rd)) {
+    if (out_host && n < cap) out_host[n] = t;
+    ++n;
+  }
+  return n;
+}
+
+}  // extern "C"

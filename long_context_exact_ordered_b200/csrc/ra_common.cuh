@@ -1,0 +1,132 @@
+// Problem description, ring-ordered KV-tile schedule and tile metadata,
+// shared by the sm_100a kernels, the CUDA-core kernels and the host.
+//
+// The ring (page "Ring Attention技术解析", §2.2): the sequence of S tokens is
+// cut into P contiguous blocks; virtual rank r owns query block r; at step t
+// it holds the key/value block that started t ranks behind it, i.e. block
+// (r - t) mod P (each rank sends its block to the next rank and receives the
+// previous rank's).  On one GPU the ranks are virtual: the ring becomes the
+// order in which a query tile visits key/value tiles.  `order` lets a caller
+// permute the steps (the result does not depend on it).
+//
+// Hardware tiles are 128 tokens.  Tile t belongs to ring block
+// floor(128 t / (S/P)) (the block of its first token), so the tiles of block
+// `src` are [ceil(src*blk/128), ceil((src+1)*blk/128)) and every tile is
+// visited exactly once.
+#pragma once
+
+#include <cstdint>
+
+#if defined(__CUDACC__)
+#define RA_HD __host__ __device__ __forceinline__
+#else
+#define RA_HD inline
+#endif
+
+namespace ra {
+
+constexpr int kTile = 128;           // tokens per hardware tile
+constexpr int kMaxRing = 64;         // largest supported ring size P
+
+struct RingDesc {
+  int64_t S;                 // sequence length (tokens)
+  int64_t blk;               // tokens per ring block, S / P
+  int32_t P;                 // ring size (virtual ranks)
+  int32_t ntiles;            // ceil(S / 128)
+  int32_t cbs;               // causal_block_size; 0 = non-causal
+  int32_t order[kMaxRing];   // step offsets t, a permutation of 0..P-1
+};
+
+// Per 128-token tile of one batch row: x = min segment id, y = max segment
+// id, z = flags (bit 0: some key has a finite bias, bit 1: every bias is 0).
+// Without segment ids x = y = 0; without a bias z = 3.
+enum : int32_t { kMetaAnyFinite = 1, kMetaAllZero = 2 };
+
+RA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+#if defined(__CUDA_ARCH__)
+RA_HD int4 load_meta(const int4* p) { return __ldg(p); }
+#else
+RA_HD int4 load_meta(const int4* p) { return *p; }
+#endif
+
+// Last key visible to any query <= q_last under causal_block_size c
+// (key j visible to query i iff floor(i/c) >= floor(j/c)).
+RA_HD int64_t causal_last_key(int64_t q_last, int32_t c, int64_t S) {
+  if (c <= 0) return S - 1;
+  int64_t j = (q_last / c + 1) * (int64_t)c - 1;
+  return j < S - 1 ? j : S - 1;
+}
+
+// Iterator over the KV tiles a query range [q_first, q_last] must visit, in
+// ring order, skipping tiles that causal masking, disjoint segment ranges or
+// an all -inf bias make invisible to every query of the range.
+struct KvIter {
+  int32_t r;          // ring block of q_first
+  int32_t step;       // current ring step
+  int32_t tile;       // next tile to consider within the step
+  int32_t tile_end;   // end of the step's tile range
+  int32_t t_cap;      // last tile not fully hidden by causal masking
+  int32_t q_seg_min, q_seg_max;
+  int32_t use_seg, use_bias;
+  const int4* meta;   // this batch row's tile metadata, or null
+};
+
+RA_HD void kv_iter_init(KvIter& it, const RingDesc& rd, int64_t q_first, int64_t q_last, const int4* meta_b,
+                        bool use_seg, bool use_bias) {
+  if (q_last > rd.S - 1) q_last = rd.S - 1;
+  it.r = (int32_t)(q_first / rd.blk);
+  it.step = -1;
+  it.tile = 0;
+  it.tile_end = 0;
+  it.t_cap = (int32_t)(causal_last_key(q_last, rd.cbs, rd.S) / kTile);
+  it.meta = (use_seg || use_bias) ? meta_b : nullptr;
+  it.use_seg = use_seg;
+  it.use_bias = use_bias;
+  it.q_seg_min = 0x7fffffff;
+  it.q_seg_max = -0x7fffffff - 1;
+  if (use_seg) {
+    for (int64_t qt = q_first / kTile; qt <= q_last / kTile; ++qt) {
+      int4 m = load_meta(meta_b + qt);
+      it.q_seg_min = m.x < it.q_seg_min ? m.x : it.q_seg_min;
+      it.q_seg_max = m.y > it.q_seg_max ? m.y : it.q_seg_max;
+    }
+  }
+}
+
+// Next KV tile index in ring order, or -1 when the ring is closed.
+RA_HD int32_t kv_iter_next(KvIter& it, const RingDesc& rd) {
+  while (true) {
+    while (it.tile < it.tile_end) {
+      int32_t t = it.tile++;
+      if (it.meta) {
+        int4 m = load_meta(it.meta + t);
+        if (it.use_seg && (m.y < it.q_seg_min || m.x > it.q_seg_max)) continue;
+        if (it.use_bias && !(m.z & kMetaAnyFinite)) continue;
+      }
+      return t;
+    }
+    if (++it.step >= rd.P) return -1;
+    int32_t src = it.r - rd.order[it.step];
+    src %= rd.P;
+    if (src < 0) src += rd.P;
+    int64_t a = (int64_t)src * rd.blk, b = (int64_t)(src + 1) * rd.blk;
+    it.tile = (int32_t)ceil_div64(a, kTile);
+    int64_t e = ceil_div64(b, kTile);
+    if (e > it.t_cap + 1) e = it.t_cap + 1;
+    it.tile_end = (int32_t)e;
+  }
+}
+
+// Whether a (query tile, KV tile) pair needs the per-element mask: a causal
+// diagonal, a partly-out-of-range KV tile, or mixed segment ids.
+RA_HD bool tile_needs_mask(const RingDesc& rd, int64_t q_first, int32_t t, bool use_seg, int4 qm, int4 km) {
+  int64_t k_first = (int64_t)t * kTile;
+  int64_t k_last = k_first + kTile - 1;
+  if (k_last > rd.S - 1) return true;
+  if (rd.cbs > 0 && (q_first / rd.cbs) < (k_last / rd.cbs)) return true;
+  if (use_seg && !(qm.x == qm.y && km.x == km.y && qm.x == km.x)) return true;
+  return false;
+}
+
+}  // namespace ra

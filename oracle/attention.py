@@ -137,15 +137,18 @@ def attention_forward(q, k, v, attention_bias=None, segment_ids=None, causal_blo
     return o, lse
 
 
-def attention_rows(q, k, v, samples, attention_bias=None, segment_ids=None, causal_block_size=None):
+def attention_rows(q, k, v, samples, attention_bias=None, segment_ids=None, causal_block_size=None,
+                   q_rows=None):
     """Forward for selected rows only.
 
     ``samples`` is an int array [n, 3] of (b, h, i).  Returns o [n, D] and
     lse [n] in the order given.  Each (b, h) head's K and V are upcast once
-    and all of its sampled rows are evaluated together.
+    and all of its sampled rows are evaluated together.  ``q_rows`` [n, D]
+    optionally supplies the sampled query vectors directly (then ``q`` is
+    not read), so a caller need not hold the whole query tensor.
     """
     samples = np.asarray(samples, dtype=np.int64).reshape(-1, 3)
-    D = np.asarray(q).shape[-1]
+    D = np.asarray(k).shape[-1]
     S = np.asarray(k).shape[1]
     o = np.zeros((len(samples), D), dtype=np.float64)
     lse = np.zeros(len(samples), dtype=np.float64)
@@ -157,7 +160,7 @@ def attention_rows(q, k, v, samples, attention_bias=None, segment_ids=None, caus
         kh, vh = _f64(k[b, :, h, :]), _f64(v[b, :, h, :])
         seg_b = None if segment_ids is None else np.asarray(segment_ids)[b]
         bias_b = None if attention_bias is None else _f64(attention_bias)[b]
-        qr = _f64(np.asarray(q)[b, rows, h, :])
+        qr = _f64(np.asarray(q)[b, rows, h, :]) if q_rows is None else _f64(np.asarray(q_rows)[idx])
         for a, e in _row_chunks(len(rows), S):
             o[idx[a:e]], lse[idx[a:e]] = _rows_forward(
                 qr[a:e], kh, vh, rows[a:e], causal_block_size, seg_b, bias_b)
