@@ -70,6 +70,13 @@ __device__ __forceinline__ bool ra_wait(uint32_t bar, uint32_t parity, volatile 
   }
 }
 
+// ra_wait for every lane of a warp, with a warp-uniform result: if any lane
+// gave up, all lanes report failure, so the warp never reaches a
+// .sync.aligned tcgen05 instruction partially.
+__device__ __forceinline__ bool ra_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, ra_wait(bar, parity, abort_flag));
+}
+
 // Bounded wait used on exit paths: ignores the abort flag (the operations it
 // waits for are already in flight and will complete), gives up only on the
 // spin budget.

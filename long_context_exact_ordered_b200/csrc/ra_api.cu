@@ -44,6 +44,15 @@ int check_tma_bf16(const ra_tensor* t) {
   return RA_OK;
 }
 
+// Output written with 16-byte vector stores (bf16 or fp32 elements).
+int check_vec16(const ra_tensor* t) {
+  const int64_t es = t->dtype == RA_BF16 ? 2 : 4;
+  if (reinterpret_cast<uintptr_t>(t->data) % 16) return RA_ERR_STRIDE;
+  for (int i = 0; i < 3; ++i)
+    if ((t->stride[i] * es) % 16) return RA_ERR_STRIDE;
+  return RA_OK;
+}
+
 // [B, H, S] fp32 (lse, m, l).
 int check_bhs(const ra_tensor* t, int64_t B, int64_t H, int64_t S) {
   if (!t) return RA_ERR_NULL;
@@ -99,8 +108,12 @@ int make_ring(const ra_params* p, int64_t S, RingDesc* rd) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Workspace layout.  Forward: tile metadata (only with bias or segment ids).
+// Backward: metadata, Delta and lse*log2(e) rows padded to a multiple of 64
+// ([B*H][s_pad] each), and the fp32 dQ accumulator [B*H][S][D].
 struct WsLayout {
-  size_t meta = 0, delta = 0, dqacc = 0, total = 0;
+  size_t meta = 0, delta = 0, lse2 = 0, dqacc = 0, total = 0;
+  int64_t s_pad = 0;
 };
 
 WsLayout ws_layout(int which, int64_t B, int64_t S, int64_t H, int64_t D, bool need_meta) {
@@ -111,8 +124,11 @@ WsLayout ws_layout(int which, int64_t B, int64_t S, int64_t H, int64_t D, bool n
     off += align256((size_t)B * ceil_div64(S, kTile) * sizeof(int4));
   }
   if (which == 1) {
+    w.s_pad = ceil_div64(S, kQTileBwd) * kQTileBwd;
     w.delta = off;
-    off += align256((size_t)B * H * S * sizeof(float));
+    off += align256((size_t)B * H * w.s_pad * sizeof(float));
+    w.lse2 = off;
+    off += align256((size_t)B * H * w.s_pad * sizeof(float));
     w.dqacc = off;
     off += align256((size_t)B * H * S * D * sizeof(float));
   }
@@ -260,6 +276,59 @@ int launch_fwd_simt(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, 
   return last_cuda();
 }
 
+int launch_bwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* d_o,
+                     const MaskArgs& mk, const RingDesc& rd, const int4* meta, const WsLayout& w, char* ws,
+                     ra_tensor* dk, ra_tensor* dv, cudaStream_t st) {
+  using L = BwdLayout;
+  CUtensorMap tq, tk, tv, tdo;
+  RA_TRY(make_tmap_bshd(&tq, q, L::QT));
+  RA_TRY(make_tmap_bshd(&tk, k, kTile));
+  RA_TRY(make_tmap_bshd(&tv, v, kTile));
+  RA_TRY(make_tmap_bshd(&tdo, d_o, L::QT));
+  BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.rd = rd;
+  prm.B = (int32_t)q->shape[0];
+  prm.H = (int32_t)q->shape[2];
+  prm.scale = (float)(1.0 / std::sqrt((double)L::D));
+  prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)L::D));
+  prm.lse2 = reinterpret_cast<const float*>(ws + w.lse2);
+  prm.delta = reinterpret_cast<const float*>(ws + w.delta);
+  prm.s_pad = w.s_pad;
+  prm.dqacc = reinterpret_cast<float*>(ws + w.dqacc);
+  prm.dk = dk->data;
+  prm.dk_sb = dk->stride[0];
+  prm.dk_ss = dk->stride[1];
+  prm.dk_sh = dk->stride[2];
+  prm.dv = dv->data;
+  prm.dv_sb = dv->stride[0];
+  prm.dv_ss = dv->stride[1];
+  prm.dv_sh = dv->stride[2];
+  prm.grad_bf16 = dk->dtype == RA_BF16;
+  prm.seg = mk.seg;
+  prm.seg_sb = mk.seg_sb;
+  prm.seg_ss = mk.seg_ss;
+  prm.bias = mk.bias;
+  prm.bias_sb = mk.bias_sb;
+  prm.bias_ss = mk.bias_ss;
+  prm.meta = meta;
+  const int64_t grid = (int64_t)rd.ntiles * prm.B * prm.H;
+  if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(ra_bwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
+      cudaSuccess)
+    return RA_ERR_CUDA;
+  ra_bwd_sm100_kernel<<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, prm);
+  return last_cuda();
+}
+
+template <int D, typename T>
+int launch_bwd_simt(const SimtBwdArgs& a, int64_t S, cudaStream_t st) {
+  dim3 grid((unsigned)ceil_div64(S, 64), (unsigned)(a.B * a.H));
+  simt_bwd_dq_kernel<D, T><<<grid, 64, 0, st>>>(a);
+  simt_bwd_dkdv_kernel<D, T><<<grid, 64, 0, st>>>(a);
+  return last_cuda();
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -364,8 +433,13 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   RingDesc rd;
   if (B * S * H == 0) return make_ring(p, S, &rd) == RA_ERR_ORDER ? RA_ERR_ORDER : RA_OK;
   RA_TRY(make_ring(p, S, &rd));
-  if (dt == RA_BF16)
+  if (dt == RA_BF16) {
     for (const ra_tensor* t : {q, k, v, o, d_o}) RA_TRY(check_tma_bf16(t));
+    if (D == 128) {
+      RA_TRY(check_vec16(dk));
+      RA_TRY(check_vec16(dv));
+    }
+  }
   const bool need_meta = attention_bias || segment_ids;
   const WsLayout w = ws_layout(1, B, S, H, D, need_meta);
   if (!workspace || workspace_bytes < w.total || reinterpret_cast<uintptr_t>(workspace) % 256)
@@ -379,20 +453,34 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   const MaskArgs mk = mask_args(attention_bias, segment_ids);
   char* ws = static_cast<char*>(workspace);
   int4* meta = need_meta ? reinterpret_cast<int4*>(ws + w.meta) : nullptr;
-  float* delta = reinterpret_cast<float*>(ws + w.delta);
-  float* dqacc = reinterpret_cast<float*>(ws + w.dqacc);
+  const bool tc_path = dt == RA_BF16 && D == 128;   // tensor-core backward; else CUDA cores
   if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
   {
-    BwdPreArgs pa{(int)B, (int)S, (int)H, (int)D, o->data, o->stride[0], o->stride[1], o->stride[2],
-                  d_o->data, d_o->stride[0], d_o->stride[1], d_o->stride[2], dt == RA_BF16, delta};
-    const int64_t threads = B * S * H * 32;
+    BwdPreArgs pa;
+    std::memset(&pa, 0, sizeof(pa));
+    pa.B = (int)B; pa.S = (int)S; pa.H = (int)H; pa.D = (int)D;
+    pa.o = o->data; pa.o_sb = o->stride[0]; pa.o_ss = o->stride[1]; pa.o_sh = o->stride[2];
+    pa.dO = d_o->data; pa.do_sb = d_o->stride[0]; pa.do_ss = d_o->stride[1]; pa.do_sh = d_o->stride[2];
+    pa.lse = static_cast<const float*>(lse->data);
+    pa.lse_sb = lse->stride[0]; pa.lse_sh = lse->stride[1]; pa.lse_ss = lse->stride[2];
+    pa.bf16 = dt == RA_BF16;
+    pa.s_pad = w.s_pad;
+    pa.delta = reinterpret_cast<float*>(ws + w.delta);
+    pa.lse2 = reinterpret_cast<float*>(ws + w.lse2);
+    pa.dqacc = tc_path ? reinterpret_cast<float*>(ws + w.dqacc) : nullptr;
+    const int64_t threads = B * H * w.s_pad * 32;
     bwd_pre_kernel<<<(unsigned)ceil_div64(threads, 256), 256, 0, st>>>(pa);
     RA_TRY(last_cuda());
   }
-  if (dt == RA_BF16) {
-    return D == 64 ? launch_bwd_sm100<64>(q, k, v, d_o, lse, mk, rd, meta, delta, dqacc, dq, dk, dv, st)
-                   : launch_bwd_sm100<128>(q, k, v, d_o, lse, mk, rd, meta, delta, dqacc, dq, dk, dv, st);
+  if (tc_path) {
+    RA_TRY(launch_bwd_sm100(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st));
+    DqConvertArgs ca{(int)B, (int)S, (int)H, (int)D, reinterpret_cast<const float*>(ws + w.dqacc),
+                     dq->data, dq->stride[0], dq->stride[1], dq->stride[2], dq->dtype == RA_BF16};
+    const int64_t n = B * S * H * D;
+    dq_convert_kernel<<<(unsigned)ceil_div64(n, 256), 256, 0, st>>>(ca);
+    return last_cuda();
   }
+  if (dk->dtype != dq->dtype || dv->dtype != dq->dtype) return RA_ERR_DTYPE;
   SimtBwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.rd = rd;
@@ -408,19 +496,14 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   a.lse_sb = lse->stride[0];
   a.lse_sh = lse->stride[1];
   a.lse_ss = lse->stride[2];
-  a.delta = delta;
+  a.delta = reinterpret_cast<const float*>(ws + w.delta);
+  a.s_pad = w.s_pad;
   a.dq = oview4(dq);
   a.dk = oview4(dk);
   a.dv = oview4(dv);
-  dim3 grid((unsigned)ceil_div64(S, 64), (unsigned)(B * H));
-  if (D == 64) {
-    simt_bwd_dq_kernel<64><<<grid, 64, 0, st>>>(a);
-    simt_bwd_dkdv_kernel<64><<<grid, 64, 0, st>>>(a);
-  } else {
-    simt_bwd_dq_kernel<128><<<grid, 64, 0, st>>>(a);
-    simt_bwd_dkdv_kernel<128><<<grid, 64, 0, st>>>(a);
-  }
-  return last_cuda();
+  a.out_bf16 = dq->dtype == RA_BF16;
+  if (dt == RA_BF16) return launch_bwd_simt<64, __nv_bfloat16>(a, S, st);
+  return D == 64 ? launch_bwd_simt<64, float>(a, S, st) : launch_bwd_simt<128, float>(a, S, st);
 }
 
 int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_blk, int64_t q_off, int64_t k_off,

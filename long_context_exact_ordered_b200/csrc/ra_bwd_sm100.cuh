@@ -1,16 +1,472 @@
-// sm_100a backward (bf16): placeholder until the tensor-core kernel lands.
+// sm_100a backward (bf16 in, fp32 accumulate, head_dim 128): gradients of
+// blockwise exact attention, recomputing probabilities from the saved
+// log-sum-exp (the recompute policy "nothing_saveable" of page
+// "RingAttention核心功能全解析", 核心API调用).
+//
+// Work unit = one (batch, head, 128-key tile).  The key/value tile stays
+// resident while 64-row query tiles stream past in ring order: in the ring,
+// a key/value block of ring block src meets query block (src + t) mod P at
+// step t (page "Ring Attention技术解析" §2.2), so dK and dV accumulate as the
+// block travels.  Per query tile i (all products on the tensor cores, fp32
+// accumulators in TMEM, M = 128 everywhere):
+//   S^T  = K Q_i^T              (SS, K-major)            -> TMEM [128 x 64]
+//   dP^T = V dO_i^T             (SS, K-major)            -> TMEM [128 x 64]
+//   P^T  = exp2(S^T log2e/sqrt(D) - lse_i log2e) (masked), dS^T = P^T (dP^T - Delta_i)
+//   dV  += P^T dO_i             (TS: P^T bf16 in TMEM, dO MN-major)
+//   dK  += dS^T Q_i             (TS: dS^T bf16 in TMEM, Q MN-major)
+//   dQ^T = K^T dS^T             (SS: K and dS^T both MN-major) -> TMEM [128 x 64]
+// dQ^T is read back by a dedicated warpgroup and reduced into an fp32
+// workspace (atomic adds; dQ gathers contributions from every key tile).
+//
+// Roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
+// warps 4-7 "softmax" (thread = key row: P^T, dS^T, final dK/dV epilogue),
+// warps 8-11 dQ readout (thread = head-dim lane d of dQ^T).
+// TMEM (512 columns): S^T [0,64) dP^T [64,128) dQ^T [128,192) P^T [192,224)
+// dS^T [224,256) dK [256,384) dV [384,512).
+//
+// Overlap: S^T(i+1), dP^T(i+1) are issued as soon as the softmax group has
+// read S^T(i), dP^T(i), ahead of dV(i), dK(i), dQ^T(i), so the softmax of
+// tile i+1 runs while the tensor core finishes tile i.
 #pragma once
 
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
 #include "ra_common.cuh"
 #include "ra_simt.cuh"
 
 namespace ra {
 
-template <int D>
-int launch_bwd_sm100(const ra_tensor*, const ra_tensor*, const ra_tensor*, const ra_tensor*, const ra_tensor*,
-                     const MaskArgs&, const RingDesc&, const int4*, float*, float*, ra_tensor*, ra_tensor*,
-                     ra_tensor*, cudaStream_t) {
-  return RA_ERR_UNSUPPORTED;
+struct BwdLayout {
+  static constexpr int D = 128;
+  static constexpr int QT = kQTileBwd;            // 64 query rows per tile
+  static constexpr int KV_BYTES = kTile * D * 2;  // 32 KB
+  static constexpr int KV_CHUNK = kTile * 128;    // 16 KB box: 128 rows x 128 B
+  static constexpr int Q_BYTES = QT * D * 2;      // 16 KB
+  static constexpr int Q_CHUNK = QT * 128;        // 8 KB box: 64 rows x 128 B
+  static constexpr int DS_BYTES = kTile * QT * 2; // 16 KB: 128 keys x 64 queries bf16
+  static constexpr int NS = 2;                    // query-side stages
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;
+  static constexpr int OFF_DO = OFF_Q + NS * Q_BYTES;
+  static constexpr int OFF_DS = OFF_DO + NS * Q_BYTES;
+  static constexpr int OFF_LD = OFF_DS + 2 * DS_BYTES;   // per stage: lse2[64], delta[64]
+  static constexpr int LD_BYTES = 2 * QT * 4;
+  static constexpr int OFF_BAR = OFF_LD + NS * LD_BYTES;
+  static constexpr int B_KV = 0;
+  static constexpr int B_QF = 1;                  // [NS]
+  static constexpr int B_QE = B_QF + NS;          // [NS]
+  static constexpr int B_SFULL = B_QE + NS;
+  static constexpr int B_DPFULL = B_SFULL + 1;
+  static constexpr int B_DSREADY = B_DPFULL + 1;
+  static constexpr int B_MMADONE = B_DSREADY + 1;
+  static constexpr int B_DQFULL = B_MMADONE + 1;
+  static constexpr int B_DQFREE = B_DQFULL + 1;
+  static constexpr int B_DSBFREE = B_DQFREE + 1;  // [2]
+  static constexpr int B_FINAL = B_DSBFREE + 2;
+  static constexpr int NBAR = B_FINAL + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DQT = 128, COL_PT = 192, COL_DST = 224, COL_DK = 256,
+                            COL_DV = 384;
+  static constexpr int THREADS = 384;
+};
+
+struct BwdParams {
+  RingDesc rd;
+  int32_t B, H;
+  float scale_log2;          // log2(e) / sqrt(D)
+  float scale;               // 1 / sqrt(D)
+  const float* lse2;         // [B*H][s_pad]: lse * log2(e), +inf for rows with no visible key
+  const float* delta;        // [B*H][s_pad]: <dO_i, O_i>
+  int64_t s_pad;
+  float* dqacc;              // [B*H][S][D] fp32, pre-zeroed
+  void* dk;
+  int64_t dk_sb, dk_ss, dk_sh;
+  void* dv;
+  int64_t dv_sb, dv_ss, dv_sh;
+  int32_t grad_bf16;         // dK / dV element type: 1 bf16, 0 fp32
+  const int32_t* seg;
+  int64_t seg_sb, seg_ss;
+  const float* bias;
+  int64_t bias_sb, bias_ss;
+  const int4* meta;
+};
+
+// 1-D bulk copy global -> shared (16-byte aligned, size multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+__global__ void __launch_bounds__(384, 1)
+    ra_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ BwdParams p) {
+  using L = BwdLayout;
+  constexpr int D = L::D;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (sbase - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // Longest units first: under causal masking the first key tiles meet the most query tiles.
+  const int BH = p.B * p.H;
+  const int kt = blockIdx.x / BH;
+  const int bh = blockIdx.x % BH;
+  const int b = bh / p.H, h = bh % p.H;
+  const int64_t k0 = (int64_t)kt * kTile;
+  const int64_t S = p.rd.S;
+
+  auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + L::OFF_MISC + 4);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(L::B_KV), 1);
+    for (int i = 0; i < L::NS; ++i) { mbar_init(bar(L::B_QF + i), 1); mbar_init(bar(L::B_QE + i), 1); }
+    mbar_init(bar(L::B_SFULL), 1);
+    mbar_init(bar(L::B_DPFULL), 1);
+    mbar_init(bar(L::B_DSREADY), 128);
+    mbar_init(bar(L::B_MMADONE), 1);
+    mbar_init(bar(L::B_DQFULL), 1);
+    mbar_init(bar(L::B_DQFREE), 128);
+    mbar_init(bar(L::B_DSBFREE + 0), 1);
+    mbar_init(bar(L::B_DSBFREE + 1), 1);
+    mbar_init(bar(L::B_FINAL), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const bool use_seg = p.seg != nullptr, use_bias = p.bias != nullptr;
+  const int4* meta_b = p.meta ? p.meta + (int64_t)b * p.rd.ntiles : nullptr;
+  const int4 km = meta_b ? load_meta(meta_b + kt) : make_int4(0, 0, 3, 0);
+  // A key tile whose every bias is -inf is invisible to all queries.
+  const bool dead = use_bias && !(km.z & kMetaAnyFinite);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_do);
+      mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::KV_BYTES);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_4d(sbase + L::OFF_K + c * L::KV_CHUNK, &tm_k, bar(L::B_KV), c * 64, h, (int)k0, b);
+        tma_load_4d(sbase + L::OFF_V + c * L::KV_CHUNK, &tm_v, bar(L::B_KV), c * 64, h, (int)k0, b);
+      }
+      int n = 0;
+      if (!dead) {
+        QIter it;
+        q_iter_init(it, p.rd, k0, meta_b, use_seg);
+        const float* lse_row = p.lse2 + (int64_t)bh * p.s_pad;
+        const float* dl_row = p.delta + (int64_t)bh * p.s_pad;
+        for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
+          const int st = n % L::NS;
+          if (n >= L::NS && !ra_wait(bar(L::B_QE + st), ((n / L::NS) & 1) ^ 1, abort_flag)) break;
+          const int q0 = q * L::QT;
+          mbar_arrive_expect_tx(bar(L::B_QF + st), 2 * L::Q_BYTES + L::LD_BYTES);
+          for (int c = 0; c < 2; ++c) {
+            tma_load_4d(sbase + L::OFF_Q + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_q, bar(L::B_QF + st), c * 64, h,
+                        q0, b);
+            tma_load_4d(sbase + L::OFF_DO + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_do, bar(L::B_QF + st), c * 64,
+                        h, q0, b);
+          }
+          bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES, lse_row + q0, L::QT * 4, bar(L::B_QF + st));
+          bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES + L::QT * 4, dl_row + q0, L::QT * 4, bar(L::B_QF + st));
+        }
+      }
+      ra_wait_drain(bar(L::B_KV), 0);
+      for (int i = n - L::NS; i < n; ++i)
+        if (i >= 0) ra_wait_drain(bar(L::B_QF + i % L::NS), (i / L::NS) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, L::QT, false, false);
+      constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, L::QT, true, true);
+      const uint32_t ka = sbase + L::OFF_K, va = sbase + L::OFF_V;
+      auto issue_sd = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {   // S^T or dP^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oa = (kk / 4) * L::KV_CHUNK + (kk % 4) * 32;
+          const uint32_t ob = (kk / 4) * L::Q_CHUNK + (kk % 4) * 32;
+          mma_ss(d_tmem, smem_desc_sw128(a_base + oa, 16, 1024), smem_desc_sw128(b_base + ob, 16, 1024), IDESC_SD,
+                 kk > 0);
+        }
+      };
+      auto issue_kv = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool acc) {   // dV or dK
+#pragma unroll
+        for (int kk = 0; kk < L::QT / 16; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_base + kk * 2048, L::Q_CHUNK, 1024), IDESC_KV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+      auto issue_dq = [&](uint32_t ds_base) {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ss(tmem + L::COL_DQT, smem_desc_sw128(ka + kk * 2048, L::KV_CHUNK, 1024),
+                 smem_desc_sw128(ds_base + kk * 2048, L::DS_BYTES, 1024), IDESC_DQ, kk > 0);
+      };
+      bool ok = ra_wait(bar(L::B_KV), 0, abort_flag);
+      if (ok && !dead) {
+        QIter it;
+        q_iter_init(it, p.rd, k0, meta_b, use_seg);
+        int32_t q = q_iter_next(it, p.rd);
+        if (q >= 0) {
+          ok = ra_wait(bar(L::B_QF + 0), 0, abort_flag);
+          if (ok) {
+            tc_fence_after();
+            issue_sd(tmem + L::COL_ST, ka, sbase + L::OFF_Q);
+            mma_commit(bar(L::B_SFULL));
+            issue_sd(tmem + L::COL_DPT, va, sbase + L::OFF_DO);
+            mma_commit(bar(L::B_DPFULL));
+          }
+          for (int n = 0; ok; ++n) {
+            const int32_t qn = q_iter_next(it, p.rd);
+            const bool last = qn < 0;
+            const int st = n % L::NS, st1 = (n + 1) % L::NS;
+            if (!(ok = ra_wait(bar(L::B_DSREADY), n & 1, abort_flag))) break;
+            tc_fence_after();
+            if (!last) {
+              if (!(ok = ra_wait(bar(L::B_QF + st1), ((n + 1) / L::NS) & 1, abort_flag))) break;
+              tc_fence_after();
+              issue_sd(tmem + L::COL_ST, ka, sbase + L::OFF_Q + st1 * L::Q_BYTES);
+              mma_commit(bar(L::B_SFULL));
+              issue_sd(tmem + L::COL_DPT, va, sbase + L::OFF_DO + st1 * L::Q_BYTES);
+              mma_commit(bar(L::B_DPFULL));
+            }
+            issue_kv(tmem + L::COL_DV, tmem + L::COL_PT, sbase + L::OFF_DO + st * L::Q_BYTES, n > 0);
+            issue_kv(tmem + L::COL_DK, tmem + L::COL_DST, sbase + L::OFF_Q + st * L::Q_BYTES, n > 0);
+            mma_commit(bar(L::B_MMADONE));
+            if (n > 0) {
+              if (!(ok = ra_wait(bar(L::B_DQFREE), (n - 1) & 1, abort_flag))) break;
+              tc_fence_after();
+            }
+            issue_dq(sbase + L::OFF_DS + (n & 1) * L::DS_BYTES);
+            mma_commit(bar(L::B_DQFULL));
+            mma_commit(bar(L::B_DSBFREE + (n & 1)));
+            mma_commit(bar(L::B_QE + st));
+            if (last) break;
+          }
+        }
+      }
+      mma_commit(bar(L::B_FINAL));
+      ra_wait_drain(bar(L::B_FINAL), 0);
+    }
+    __syncwarp();
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ softmax group: one key row per thread
+    const int sub = warp & 3;
+    const int row = sub * 32 + lane;
+    const int64_t j = k0 + row;                      // this thread's key
+    const bool row_valid = j < S;
+    const int64_t jc = row_valid ? j : S - 1;
+    const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
+    const uint32_t trow = tmem + lane_off;
+    const int my_seg = use_seg ? p.seg[b * p.seg_sb + jc * p.seg_ss] : 0;
+    float brow = 0.f;                                // bias of this key, log2 units
+    if (use_bias) brow = p.bias[b * p.bias_sb + jc * p.bias_ss] * kLog2e;
+    const int32_t cbs = p.rd.cbs;
+    const int64_t i_first = cbs > 0 ? (j / cbs) * (int64_t)cbs : 0;   // first query that can see key j
+    int n = 0;
+    bool ok = true;
+    if (!dead) {
+      QIter it;
+      q_iter_init(it, p.rd, k0, meta_b, use_seg);
+      for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
+        const int st = n % L::NS;
+        const int64_t q0 = (int64_t)q * L::QT;
+        if (!(ok = ra_wait_warp(bar(L::B_QF + st), (n / L::NS) & 1, abort_flag))) break;
+        if (!(ok = ra_wait_warp(bar(L::B_SFULL), n & 1, abort_flag))) break;
+        tc_fence_after();
+        uint32_t sr[64];
+        tmem_ld32(trow + L::COL_ST, sr);
+        tmem_ld32(trow + L::COL_ST + 32, sr + 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 64; ++c) reg_fence(sr[c]);
+        float* x = reinterpret_cast<float*>(sr);
+        const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + st * L::LD_BYTES);
+        const float* dlt = lse2 + L::QT;
+#pragma unroll
+        for (int c = 0; c < 64; ++c) x[c] = fmaf(x[c], p.scale_log2, brow - lse2[c]);
+        // per-element mask on causal-diagonal / ragged / mixed-segment tiles
+        const int4 qm = meta_b ? load_meta(meta_b + q0 / kTile) : make_int4(0, 0, 3, 0);
+        const bool need_causal = cbs > 0 && (q0 / cbs) < ((k0 + kTile - 1) / cbs);
+        const bool need_ragged = (q0 + L::QT > S) || (k0 + kTile > S);
+        const bool need_seg = use_seg && !(qm.x == qm.y && km.x == km.y && qm.x == km.x);
+        if (need_causal || need_ragged || need_seg || !row_valid) {
+          const int64_t cmin64 = i_first - q0;                   // visible iff c >= cmin
+          const int cmin = cmin64 < 0 ? 0 : (cmin64 > 64 ? 64 : (int)cmin64);
+          const int64_t cmax64 = S - q0;                         // valid iff c < cmax
+          const int cmax = row_valid ? (cmax64 > 64 ? 64 : (int)cmax64) : 0;
+          uint32_t vb0 = ~0u, vb1 = ~0u;
+          if (need_seg) {
+            const int32_t* sp = p.seg + b * p.seg_sb;
+            vb0 = 0;
+            vb1 = 0;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int64_t i = q0 + c < S ? q0 + c : S - 1;
+              vb0 |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << c;
+            }
+            asm volatile("" ::: "memory");
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int64_t i = q0 + 32 + c < S ? q0 + 32 + c : S - 1;
+              vb1 |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << c;
+            }
+          }
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const uint32_t bit = c < 32 ? (vb0 >> c) & 1u : (vb1 >> (c - 32)) & 1u;
+            const bool vis = c >= cmin && c < cmax && bit;
+            x[c] = vis ? x[c] : -INFINITY;
+          }
+        }
+        float pr[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) pr[c] = ex2_approx(x[c]);
+        if (!(ok = ra_wait_warp(bar(L::B_DPFULL), n & 1, abort_flag))) break;
+        tc_fence_after();
+        uint32_t dr[64];
+        tmem_ld32(trow + L::COL_DPT, dr);
+        tmem_ld32(trow + L::COL_DPT + 32, dr + 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 64; ++c) reg_fence(dr[c]);
+        uint32_t pp[32], dd[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          const float ds0 = pr[c] * (__uint_as_float(dr[c]) - dlt[c]);
+          const float ds1 = pr[c + 1] * (__uint_as_float(dr[c + 1]) - dlt[c + 1]);
+          pp[c >> 1] = pack_bf16x2(pr[c], pr[c + 1]);
+          dd[c >> 1] = pack_bf16x2(ds0, ds1);
+        }
+        // P^T / dS^T columns of TMEM are free once dV(n-1), dK(n-1) completed
+        if (n > 0 && !(ok = ra_wait_warp(bar(L::B_MMADONE), (n - 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        tmem_st32(trow + L::COL_PT, pp);
+        tmem_st32(trow + L::COL_DST, dd);
+        // dS^T into shared memory for dQ^T = K^T dS^T (MN-major, 128-byte swizzle):
+        // key row `row` is one 128-byte line; 16-byte chunk c lands at c ^ (row % 8).
+        const int buf = n & 1;
+        if (n >= 2 && !(ok = ra_wait_warp(bar(L::B_DSBFREE + buf), ((n >> 1) - 1) & 1, abort_flag))) break;
+        const uint32_t line = sbase + L::OFF_DS + buf * L::DS_BYTES + row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(line + ((c ^ (row & 7)) << 4), dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_DSREADY));
+      }
+    }
+    // ---------------------------------------------------------- dK / dV epilogue
+    bool have = n > 0 && ok;
+    if (have) have = ra_wait(bar(L::B_FINAL), 0, abort_flag);
+    have = __all_sync(0xffffffffu, have);
+    n = __shfl_sync(0xffffffffu, n, 0);
+    tc_fence_after();
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t col = which == 0 ? L::COL_DK : L::COL_DV;
+      const float mul = which == 0 ? p.scale : 1.f;
+      char* base = static_cast<char*>(which == 0 ? p.dk : p.dv);
+      const int64_t sb = which == 0 ? p.dk_sb : p.dv_sb, ss = which == 0 ? p.dk_ss : p.dv_ss,
+                    sh = which == 0 ? p.dk_sh : p.dv_sh;
+      const int64_t off = b * sb + jc * ss + h * sh;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t r[32];
+        if (have) {
+          tmem_ld32(trow + col + c, r);
+          tmem_ld_wait();
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          if (have) reg_fence(r[e]);
+          else r[e] = 0u;
+        }
+        if (row_valid && (have || n == 0)) {
+          if (p.grad_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + off + c);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                w[e] = pack_bf16x2(__uint_as_float(r[8 * v4 + 2 * e]) * mul, __uint_as_float(r[8 * v4 + 2 * e + 1]) * mul);
+              dst[v4] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + off + c);
+#pragma unroll
+            for (int v4 = 0; v4 < 8; ++v4)
+              dst[v4] = make_float4(__uint_as_float(r[4 * v4]) * mul, __uint_as_float(r[4 * v4 + 1]) * mul,
+                                    __uint_as_float(r[4 * v4 + 2]) * mul, __uint_as_float(r[4 * v4 + 3]) * mul);
+          }
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ readout: thread = head-dim lane d
+    const int sub = warp & 3;
+    const int d = sub * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16) + L::COL_DQT;
+    if (!dead) {
+      QIter it;
+      q_iter_init(it, p.rd, k0, meta_b, use_seg);
+      int n = 0;
+      for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
+        if (!ra_wait_warp(bar(L::B_DQFULL), n & 1, abort_flag)) break;
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld32(trow, r);
+        tmem_ld32(trow + 32, r + 32);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 64; ++c) reg_fence(r[c]);
+        tc_fence_before();
+        mbar_arrive(bar(L::B_DQFREE));
+        const int64_t q0 = (int64_t)q * L::QT;
+        float* dst = p.dqacc + ((int64_t)bh * S + q0) * D + d;
+        const int64_t nvalid = S - q0;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c < nvalid) atomicAdd(dst + (int64_t)c * D, __uint_as_float(r[c]) * p.scale);
+      }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
 }
 
 }  // namespace ra

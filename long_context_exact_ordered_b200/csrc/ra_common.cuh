@@ -26,6 +26,8 @@
 namespace ra {
 
 constexpr int kTile = 128;           // tokens per hardware tile
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kMaxRing = 64;         // largest supported ring size P
 
 struct RingDesc {
@@ -115,6 +117,63 @@ RA_HD int32_t kv_iter_next(KvIter& it, const RingDesc& rd) {
     int64_t e = ceil_div64(b, kTile);
     if (e > it.t_cap + 1) e = it.t_cap + 1;
     it.tile_end = (int32_t)e;
+  }
+}
+
+// Backward direction of the same ring: a key/value tile of ring block src
+// meets the query blocks (src + order[t]) mod P at steps t = 0, 1, ...
+// (rank r holds block (r - order[t]) mod P at step t).  QIter walks the
+// 64-row query tiles a key tile [k_first, k_last] must visit in that order,
+// skipping tiles hidden from it by causal masking or disjoint segments.
+constexpr int kQTileBwd = 64;
+
+struct QIter {
+  int32_t src;        // ring block of the key tile
+  int32_t step;
+  int32_t tile, tile_end;
+  int32_t q_min;      // first query tile not fully hidden by causal masking
+  int32_t nqt;        // number of 64-row query tiles
+  int32_t k_seg_min, k_seg_max;
+  int32_t use_seg;
+  const int4* meta;   // 128-token tile metadata of this batch row, or null
+};
+
+RA_HD void q_iter_init(QIter& it, const RingDesc& rd, int64_t k_first, const int4* meta_b, bool use_seg) {
+  it.src = (int32_t)(k_first / rd.blk);
+  it.step = -1;
+  it.tile = it.tile_end = 0;
+  it.nqt = (int32_t)ceil_div64(rd.S, kQTileBwd);
+  const int64_t i_min = rd.cbs > 0 ? (k_first / rd.cbs) * (int64_t)rd.cbs : 0;   // first query that can see k_first's block
+  it.q_min = (int32_t)(i_min / kQTileBwd);
+  it.use_seg = use_seg;
+  it.meta = use_seg ? meta_b : nullptr;
+  it.k_seg_min = 0;
+  it.k_seg_max = 0;
+  if (use_seg) {
+    int4 m = load_meta(meta_b + k_first / kTile);
+    it.k_seg_min = m.x;
+    it.k_seg_max = m.y;
+  }
+}
+
+RA_HD int32_t q_iter_next(QIter& it, const RingDesc& rd) {
+  while (true) {
+    while (it.tile < it.tile_end) {
+      int32_t q = it.tile++;
+      if (it.meta) {
+        int4 m = load_meta(it.meta + (int64_t)q * kQTileBwd / kTile);
+        if (m.y < it.k_seg_min || m.x > it.k_seg_max) continue;
+      }
+      return q;
+    }
+    if (++it.step >= rd.P) return -1;
+    int32_t r = (it.src + rd.order[it.step]) % rd.P;
+    int64_t a = (int64_t)r * rd.blk, b = (int64_t)(r + 1) * rd.blk;
+    int64_t lo = ceil_div64(a, kQTileBwd), hi = ceil_div64(b, kQTileBwd);
+    if (hi > it.nqt) hi = it.nqt;
+    if (lo < it.q_min) lo = it.q_min;
+    it.tile = (int32_t)lo;
+    it.tile_end = (int32_t)(hi > lo ? hi : lo);
   }
 }
 

@@ -92,8 +92,6 @@ struct FwdParams {
   const int4* meta;        // [B, ntiles] or null
 };
 
-constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 template <int D>
@@ -287,7 +285,7 @@ __global__ void __launch_bounds__(384, 1)
     int n = 0;
     bool ok = true;
     for (int32_t t = kv_iter_next(it, p.rd); t >= 0; t = kv_iter_next(it, p.rd), ++n) {
-      if (!(ok = ra_wait(bar(L::B_SFULL + qt), n & 1, abort_flag))) break;
+      if (!(ok = ra_wait_warp(bar(L::B_SFULL + qt), n & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld32(tS_row + 0, sr);
@@ -398,7 +396,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive(bar(L::B_PFULL + qt));
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && n > 0) ok = ra_wait(bar(L::B_PVDONE + qt), (n - 1) & 1, abort_flag);
+    if (ok && n > 0) ok = ra_wait_warp(bar(L::B_PVDONE + qt), (n - 1) & 1, abort_flag);
+    n = __shfl_sync(0xffffffffu, n, 0);   // warp-uniform (lanes agree unless a wait gave up)
     tc_fence_after();
     const float inv = l > 0.f ? 1.f / l : 0.f;
     __nv_bfloat16* op = p.o + b * p.o_sb + qrow_c * p.o_ss + h * p.o_sh;

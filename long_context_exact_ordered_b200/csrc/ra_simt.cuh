@@ -405,19 +405,34 @@ struct BwdPreArgs {
   int B, S, H, D;
   const void* o; int64_t o_sb, o_ss, o_sh;
   const void* dO; int64_t do_sb, do_ss, do_sh;
+  const float* lse; int64_t lse_sb, lse_sh, lse_ss;
   int bf16;
-  float* delta;          // [B, H, S] contiguous
+  int64_t s_pad;
+  float* delta;          // [B*H][s_pad]
+  float* lse2;           // [B*H][s_pad]
+  float* dqacc;          // [B*H][S][D] or null
 };
 
-// Backward preprocess: Delta_i = <dO_i, O_i> in fp32.  One warp per row.
+// Backward preprocess, one warp per (b, h, i) row of the padded [B*H][s_pad]
+// layout: Delta_i = <dO_i, O_i> (fp32), lse2_i = lse_i * log2(e) (+inf for a
+// row with no visible key, so its probabilities come out as 0), and the row
+// of the fp32 dQ accumulator set to zero.  Padding rows get Delta = 0 and
+// lse2 = +inf.
 __global__ void bwd_pre_kernel(const BwdPreArgs a) {
   const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t n = (int64_t)a.B * a.S * a.H;
+  const int64_t n = (int64_t)a.B * a.H * a.s_pad;
   if (row >= n) return;
-  const int h = (int)(row % a.H);
-  const int64_t i = (row / a.H) % a.S;
-  const int b = (int)(row / ((int64_t)a.H * a.S));
+  const int64_t i = row % a.s_pad;
+  const int64_t bh = row / a.s_pad;
+  const int h = (int)(bh % a.H), b = (int)(bh / a.H);
+  if (i >= a.S) {
+    if (lane == 0) {
+      a.delta[row] = 0.f;
+      a.lse2[row] = CUDART_INF_F;
+    }
+    return;
+  }
   float s = 0.f;
   const int64_t io = b * a.o_sb + i * a.o_ss + h * a.o_sh;
   const int64_t id = b * a.do_sb + i * a.do_ss + h * a.do_sh;
@@ -428,9 +443,36 @@ __global__ void bwd_pre_kernel(const BwdPreArgs a) {
     } else {
       s += static_cast<const float*>(a.o)[io + e] * static_cast<const float*>(a.dO)[id + e];
     }
+    if (a.dqacc) a.dqacc[(bh * a.S + i) * a.D + e] = 0.f;
   }
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-  if (lane == 0) a.delta[((int64_t)b * a.H + h) * a.S + i] = s;
+  if (lane == 0) {
+    a.delta[row] = s;
+    const float l = a.lse[b * a.lse_sb + h * a.lse_sh + i * a.lse_ss];
+    a.lse2[row] = l == -CUDART_INF_F ? CUDART_INF_F : l * 1.4426950408889634f;
+  }
+}
+
+struct DqConvertArgs {
+  int B, S, H, D;
+  const float* dqacc;    // [B*H][S][D]
+  void* dq; int64_t dq_sb, dq_ss, dq_sh;
+  int bf16;
+};
+
+// dQ accumulator (fp32, [B*H][S][D]) -> dq [B, S, H, D] in bf16 or fp32.
+__global__ void dq_convert_kernel(const DqConvertArgs a) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t n = (int64_t)a.B * a.S * a.H * a.D;
+  if (idx >= n) return;
+  const int e = (int)(idx % a.D);
+  const int64_t i = (idx / a.D) % a.S;
+  const int64_t bh = idx / ((int64_t)a.D * a.S);
+  const int h = (int)(bh % a.H), b = (int)(bh / a.H);
+  const float x = a.dqacc[idx];
+  const int64_t o = b * a.dq_sb + i * a.dq_ss + h * a.dq_sh + e;
+  if (a.bf16) static_cast<__nv_bfloat16*>(a.dq)[o] = __float2bfloat16_rn(x);
+  else static_cast<float*>(a.dq)[o] = x;
 }
 
 struct SimtBwdArgs {
@@ -440,8 +482,10 @@ struct SimtBwdArgs {
   MaskArgs mk;
   View4 q, k, v, dO;
   const float* lse; int64_t lse_sb, lse_sh, lse_ss;
-  const float* delta;    // [B, H, S]
+  const float* delta;    // [B*H][s_pad]
+  int64_t s_pad;
   OutView4 dq, dk, dv;
+  int out_bf16;          // gradient element type: 1 bf16, 0 fp32
 };
 
 __device__ __forceinline__ bool simt_visible(const SimtBwdArgs& a, int b, int64_t i, int64_t j, float& bias_j) {
@@ -456,17 +500,26 @@ __device__ __forceinline__ bool simt_visible(const SimtBwdArgs& a, int b, int64_
   return true;
 }
 
-// dQ for fp32 inputs: one thread per query row, keys visited in ring order.
+__device__ __forceinline__ void simt_store_row(const OutView4& o, int b, int64_t i, int h, const float* x, int D,
+                                               int bf16) {
+  const int64_t off = b * o.sb + i * o.ss + h * o.sh;
+  for (int e = 0; e < D; ++e) {
+    if (bf16) static_cast<__nv_bfloat16*>(o.p)[off + e] = __float2bfloat16_rn(x[e]);
+    else static_cast<float*>(o.p)[off + e] = x[e];
+  }
+}
+
+// dQ on CUDA cores: one thread per query row, keys visited in ring order.
 // grid (ceil(S/64), B*H), block 64.
-template <int D>
+template <int D, typename T>
 __global__ void __launch_bounds__(64) simt_bwd_dq_kernel(const SimtBwdArgs a) {
   const int b = blockIdx.y / a.H, h = blockIdx.y % a.H;
   const int64_t i = (int64_t)blockIdx.x * 64 + threadIdx.x;
   if (i >= a.rd.S) return;
-  const float* q = static_cast<const float*>(a.q.p) + b * a.q.sb + i * a.q.ss + h * a.q.sh;
-  const float* dO = static_cast<const float*>(a.dO.p) + b * a.dO.sb + i * a.dO.ss + h * a.dO.sh;
+  const T* q = static_cast<const T*>(a.q.p) + b * a.q.sb + i * a.q.ss + h * a.q.sh;
+  const T* dO = static_cast<const T*>(a.dO.p) + b * a.dO.sb + i * a.dO.ss + h * a.dO.sh;
   const float lse = a.lse[b * a.lse_sb + h * a.lse_sh + i * a.lse_ss];
-  const float dl = a.delta[((int64_t)b * a.H + h) * a.rd.S + i];
+  const float dl = a.delta[(int64_t)blockIdx.y * a.s_pad + i];
   float acc[D];
 #pragma unroll
   for (int e = 0; e < D; ++e) acc[e] = 0.f;
@@ -477,33 +530,31 @@ __global__ void __launch_bounds__(64) simt_bwd_dq_kernel(const SimtBwdArgs a) {
       for (int64_t j = (int64_t)t * kTile; j < min64(a.rd.S, (int64_t)t * kTile + kTile); ++j) {
         float bj;
         if (!simt_visible(a, b, i, j, bj)) continue;
-        const float* k = static_cast<const float*>(a.k.p) + b * a.k.sb + j * a.k.ss + h * a.k.sh;
-        const float* v = static_cast<const float*>(a.v.p) + b * a.v.sb + j * a.v.ss + h * a.v.sh;
+        const T* k = static_cast<const T*>(a.k.p) + b * a.k.sb + j * a.k.ss + h * a.k.sh;
+        const T* v = static_cast<const T*>(a.v.p) + b * a.v.sb + j * a.v.ss + h * a.v.sh;
         float s = 0.f, dp = 0.f;
         for (int e = 0; e < D; ++e) {
-          s = fmaf(q[e], k[e], s);
-          dp = fmaf(dO[e], v[e], dp);
+          s = fmaf(to_f<T>(q[e]), to_f<T>(k[e]), s);
+          dp = fmaf(to_f<T>(dO[e]), to_f<T>(v[e]), dp);
         }
         const float p = expf(s * a.scale + bj - lse);
         const float ds = p * (dp - dl) * a.scale;
 #pragma unroll
-        for (int e = 0; e < D; ++e) acc[e] = fmaf(ds, k[e], acc[e]);
+        for (int e = 0; e < D; ++e) acc[e] = fmaf(ds, to_f<T>(k[e]), acc[e]);
       }
     }
   }
-  float* out = static_cast<float*>(a.dq.p) + b * a.dq.sb + i * a.dq.ss + h * a.dq.sh;
-#pragma unroll
-  for (int e = 0; e < D; ++e) out[e] = acc[e];
+  simt_store_row(a.dq, b, i, h, acc, D, a.out_bf16);
 }
 
-// dK, dV for fp32 inputs: one thread per key row, all query rows visited.
-template <int D>
+// dK, dV on CUDA cores: one thread per key row, all query rows visited.
+template <int D, typename T>
 __global__ void __launch_bounds__(64) simt_bwd_dkdv_kernel(const SimtBwdArgs a) {
   const int b = blockIdx.y / a.H, h = blockIdx.y % a.H;
   const int64_t j = (int64_t)blockIdx.x * 64 + threadIdx.x;
   if (j >= a.rd.S) return;
-  const float* k = static_cast<const float*>(a.k.p) + b * a.k.sb + j * a.k.ss + h * a.k.sh;
-  const float* v = static_cast<const float*>(a.v.p) + b * a.v.sb + j * a.v.ss + h * a.v.sh;
+  const T* k = static_cast<const T*>(a.k.p) + b * a.k.sb + j * a.k.ss + h * a.k.sh;
+  const T* v = static_cast<const T*>(a.v.p) + b * a.v.sb + j * a.v.ss + h * a.v.sh;
   float dk[D], dv[D];
 #pragma unroll
   for (int e = 0; e < D; ++e) { dk[e] = 0.f; dv[e] = 0.f; }
@@ -512,25 +563,23 @@ __global__ void __launch_bounds__(64) simt_bwd_dkdv_kernel(const SimtBwdArgs a) 
     if (!simt_visible(a, b, i, j, bj)) continue;
     const float lse = a.lse[b * a.lse_sb + h * a.lse_sh + i * a.lse_ss];
     if (!(lse > -CUDART_INF_F)) continue;
-    const float* q = static_cast<const float*>(a.q.p) + b * a.q.sb + i * a.q.ss + h * a.q.sh;
-    const float* dO = static_cast<const float*>(a.dO.p) + b * a.dO.sb + i * a.dO.ss + h * a.dO.sh;
+    const T* q = static_cast<const T*>(a.q.p) + b * a.q.sb + i * a.q.ss + h * a.q.sh;
+    const T* dO = static_cast<const T*>(a.dO.p) + b * a.dO.sb + i * a.dO.ss + h * a.dO.sh;
     float s = 0.f, dp = 0.f;
     for (int e = 0; e < D; ++e) {
-      s = fmaf(q[e], k[e], s);
-      dp = fmaf(dO[e], v[e], dp);
+      s = fmaf(to_f<T>(q[e]), to_f<T>(k[e]), s);
+      dp = fmaf(to_f<T>(dO[e]), to_f<T>(v[e]), dp);
     }
     const float p = expf(s * a.scale + bj - lse);
-    const float ds = p * (dp - a.delta[((int64_t)b * a.H + h) * a.rd.S + i]) * a.scale;
+    const float ds = p * (dp - a.delta[(int64_t)blockIdx.y * a.s_pad + i]) * a.scale;
 #pragma unroll
     for (int e = 0; e < D; ++e) {
-      dv[e] = fmaf(p, dO[e], dv[e]);
-      dk[e] = fmaf(ds, q[e], dk[e]);
+      dv[e] = fmaf(p, to_f<T>(dO[e]), dv[e]);
+      dk[e] = fmaf(ds, to_f<T>(q[e]), dk[e]);
     }
   }
-  float* ok = static_cast<float*>(a.dk.p) + b * a.dk.sb + j * a.dk.ss + h * a.dk.sh;
-  float* ov = static_cast<float*>(a.dv.p) + b * a.dv.sb + j * a.dv.ss + h * a.dv.sh;
-#pragma unroll
-  for (int e = 0; e < D; ++e) { ok[e] = dk[e]; ov[e] = dv[e]; }
+  simt_store_row(a.dk, b, j, h, dk, D, a.out_bf16);
+  simt_store_row(a.dv, b, j, h, dv, D, a.out_bf16);
 }
 
 }  // namespace ra

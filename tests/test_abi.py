@@ -122,9 +122,9 @@ def test_workspace_size_layout():
     assert lib.ra_workspace_size(0, ctypes.byref(q), ctypes.byref(p), 0, 0) == 0
     meta = ((2 * 8 * 16 + 255) // 256) * 256      # 8 tiles of 128 tokens per batch row
     assert lib.ra_workspace_size(0, ctypes.byref(q), ctypes.byref(p), 1, 0) == meta
-    delta = ((2 * 3 * 1000 * 4 + 255) // 256) * 256
+    rows = 2 * 3 * 1024 * 4                        # Delta and lse rows padded to a multiple of 64
     dq = ((2 * 3 * 1000 * 128 * 4 + 255) // 256) * 256
-    assert lib.ra_workspace_size(1, ctypes.byref(q), ctypes.byref(p), 0, 1) == meta + delta + dq
+    assert lib.ra_workspace_size(1, ctypes.byref(q), ctypes.byref(p), 0, 1) == meta + 2 * rows + dq
     assert lib.ra_workspace_size(2, ctypes.byref(q), ctypes.byref(p), 0, 0) == ctypes.c_size_t(-1).value
 
 
