@@ -94,6 +94,12 @@ typedef struct {
   int32_t ring_order[RA_MAX_RING];
   int32_t use_ring_order;
   int32_t reserved;   /* must be 0 */
+  /* Optional profiling hooks: two cudaEvent_t handles (or NULL).  When both
+   * are set, ra_forward / ra_backward record them on `stream` immediately
+   * before and after their main attention kernel, so a caller can time that
+   * kernel alone (preprocessing and conversion launches excluded). */
+  void* prof_event_begin;
+  void* prof_event_end;
 } ra_params;
 
 /* Workspace bytes (device memory, caller-allocated, 256-byte aligned base)

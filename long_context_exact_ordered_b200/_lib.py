@@ -40,6 +40,8 @@ class RaParams(ctypes.Structure):
         ("ring_order", ctypes.c_int32 * RA_MAX_RING),
         ("use_ring_order", ctypes.c_int32),
         ("reserved", ctypes.c_int32),
+        ("prof_event_begin", ctypes.c_void_p),
+        ("prof_event_end", ctypes.c_void_p),
     ]
 
 

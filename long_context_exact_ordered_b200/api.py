@@ -37,8 +37,15 @@ def _ref(x):
     return None if x is None else ctypes.byref(x)
 
 
-def _params(S: int, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order) -> RaParams:
+def _params(S: int, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order,
+            prof_events=None) -> RaParams:
     p = RaParams()
+    if prof_events is not None:
+        for ev in prof_events:
+            if not ev.cuda_event:      # torch creates the CUDA event lazily, on its first record
+                ev.record()
+        p.prof_event_begin = prof_events[0].cuda_event
+        p.prof_event_end = prof_events[1].cuda_event
     blk = max(1, S // max(1, ring_size))
     p.query_chunk_size = blk if query_chunk_size is None else int(query_chunk_size)
     p.key_chunk_size = blk if key_chunk_size is None else int(key_chunk_size)
@@ -73,7 +80,8 @@ def _workspace(nbytes: int, device) -> torch.Tensor | None:
 
 
 def ringattention(q, k, v, attention_bias=None, segment_ids=None, query_chunk_size=512, key_chunk_size=512,
-                  causal_block_size=None, ring_size=1, ring_order=None, out=None, lse=None, workspace=None):
+                  causal_block_size=None, ring_size=1, ring_order=None, out=None, lse=None, workspace=None,
+                  prof_events=None):
     """Exact attention over ``ring_size`` virtual ring ranks.  Returns (o, lse).
 
     q, k, v: [B, S, H, D] bf16 (tensor-core path) or fp32 (CUDA-core path),
@@ -82,9 +90,11 @@ def ringattention(q, k, v, attention_bias=None, segment_ids=None, query_chunk_si
     causal_block_size: None/0 non-causal, c >= 1 block-causal.
     Chunk sizes must divide S / ring_size (they group the kernels' tiles and
     do not change the result); ``None`` means one chunk per ring block.
+    ``prof_events``: optional (begin, end) torch.cuda.Event pair recorded
+    around the main kernel only.
     """
     B, S, H, D = q.shape
-    p = _params(S, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order)
+    p = _params(S, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order, prof_events)
     if out is None:
         out = torch.empty_like(q, memory_format=torch.contiguous_format)
     if lse is None:
@@ -103,18 +113,23 @@ def ringattention(q, k, v, attention_bias=None, segment_ids=None, query_chunk_si
 
 def ringattention_backward(q, k, v, o, lse, do, attention_bias=None, segment_ids=None, query_chunk_size=512,
                            key_chunk_size=512, causal_block_size=None, ring_size=1, ring_order=None,
-                           grad_dtype=None, workspace=None):
+                           grad_dtype=None, workspace=None, out=None, prof_events=None):
     """Gradients (dq, dk, dv) of ringattention given the upstream ``do``.
 
     Recomputes attention from q, k and the saved ``lse``.  ``grad_dtype``
     defaults to the input dtype (bf16 gradients may be requested as fp32).
+    ``out``: optional preallocated (dq, dk, dv); ``prof_events`` as in
+    ringattention.
     """
     B, S, H, D = q.shape
-    p = _params(S, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order)
+    p = _params(S, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order, prof_events)
     gd = q.dtype if grad_dtype is None else grad_dtype
-    dq = torch.empty(q.shape, dtype=gd, device=q.device)
-    dk = torch.empty(q.shape, dtype=gd, device=q.device)
-    dv = torch.empty(q.shape, dtype=gd, device=q.device)
+    if out is not None:
+        dq, dk, dv = out
+    else:
+        dq = torch.empty(q.shape, dtype=gd, device=q.device)
+        dk = torch.empty(q.shape, dtype=gd, device=q.device)
+        dv = torch.empty(q.shape, dtype=gd, device=q.device)
     need = workspace_size(1, q, p, attention_bias is not None, segment_ids is not None)
     if workspace is None or workspace.numel() < need:
         workspace = _workspace(need, q.device)

@@ -180,6 +180,20 @@ int make_tmap_bshd(CUtensorMap* m, const ra_tensor* t, int rows) {
 
 int last_cuda() { return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA; }
 
+// Profiling hooks of ra_params: events recorded around the main kernel.
+struct ProfScope {
+  cudaEvent_t b = nullptr, e = nullptr;
+  cudaStream_t st;
+  ProfScope(const ra_params* p, cudaStream_t s) : st(s) {
+    if (p && p->prof_event_begin && p->prof_event_end) {
+      b = static_cast<cudaEvent_t>(p->prof_event_begin);
+      e = static_cast<cudaEvent_t>(p->prof_event_end);
+    }
+  }
+  void begin() const { if (b) cudaEventRecord(b, st); }
+  void end() const { if (e) cudaEventRecord(e, st); }
+};
+
 MaskArgs mask_args(const ra_tensor* bias, const ra_tensor* seg) {
   MaskArgs mk{};
   if (seg) {
@@ -400,12 +414,18 @@ int ra_forward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const
   const MaskArgs mk = mask_args(attention_bias, segment_ids);
   int4* meta = need_meta ? reinterpret_cast<int4*>(static_cast<char*>(workspace) + w.meta) : nullptr;
   if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
+  const ProfScope prof(p, st);
+  prof.begin();
+  int rc;
   if (dt == RA_BF16) {
-    return D == 64 ? launch_fwd_sm100<64>(q, k, v, mk, rd, meta, o, lse, st)
-                   : launch_fwd_sm100<128>(q, k, v, mk, rd, meta, o, lse, st);
-  }
-  return D == 64 ? launch_fwd_simt<64, float>(q, k, v, mk, rd, meta, o, lse, st)
+    rc = D == 64 ? launch_fwd_sm100<64>(q, k, v, mk, rd, meta, o, lse, st)
+                 : launch_fwd_sm100<128>(q, k, v, mk, rd, meta, o, lse, st);
+  } else {
+    rc = D == 64 ? launch_fwd_simt<64, float>(q, k, v, mk, rd, meta, o, lse, st)
                  : launch_fwd_simt<128, float>(q, k, v, mk, rd, meta, o, lse, st);
+  }
+  prof.end();
+  return rc;
 }
 
 int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* o,
@@ -472,8 +492,12 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
     bwd_pre_kernel<<<(unsigned)ceil_div64(threads, 256), 256, 0, st>>>(pa);
     RA_TRY(last_cuda());
   }
+  const ProfScope prof(p, st);
   if (tc_path) {
-    RA_TRY(launch_bwd_sm100(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st));
+    prof.begin();
+    const int rc = launch_bwd_sm100(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st);
+    prof.end();
+    RA_TRY(rc);
     DqConvertArgs ca{(int)B, (int)S, (int)H, (int)D, reinterpret_cast<const float*>(ws + w.dqacc),
                      dq->data, dq->stride[0], dq->stride[1], dq->stride[2], dq->dtype == RA_BF16};
     const int64_t n = B * S * H * D;
@@ -502,8 +526,12 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   a.dk = oview4(dk);
   a.dv = oview4(dv);
   a.out_bf16 = dq->dtype == RA_BF16;
-  if (dt == RA_BF16) return launch_bwd_simt<64, __nv_bfloat16>(a, S, st);
-  return D == 64 ? launch_bwd_simt<64, float>(a, S, st) : launch_bwd_simt<128, float>(a, S, st);
+  prof.begin();
+  int rc;
+  if (dt == RA_BF16) rc = launch_bwd_simt<64, __nv_bfloat16>(a, S, st);
+  else rc = D == 64 ? launch_bwd_simt<64, float>(a, S, st) : launch_bwd_simt<128, float>(a, S, st);
+  prof.end();
+  return rc;
 }
 
 int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_blk, int64_t q_off, int64_t k_off,

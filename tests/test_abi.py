@@ -36,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 def test_struct_layout_matches_header():
     assert ctypes.sizeof(_lib.RaTensor) == 8 + 4 + 4 + 32 + 32
-    assert ctypes.sizeof(_lib.RaParams) == 4 * 8 + 64 * 4 + 8
+    assert ctypes.sizeof(_lib.RaParams) == 4 * 8 + 64 * 4 + 8 + 2 * 8
 
 
 def test_strerror_covers_codes():

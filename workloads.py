@@ -17,6 +17,7 @@ packed128k     1   32  128  131072     8  512    1       bf16 N(0,1), packed doc
 causal128k     1   32  128  131072     8  512    1       bf16 N(0,1) (+dO)
 causal64k      1   32  128  65536      8  512    1       bf16 N(0,1) + dO, fwd+bwd
 causal1m       1   32  128  1048576    8  512    1       bf16 N(0,1)/sqrt(128)
+causal16k      1   32  128  16384      8  512    1       bf16 N(0,1) + dO (profiling)
 =============  ==  ==  ===  =========  =  =====  ======  ========================
 
 Random tensors: ``torch.Generator(device).manual_seed(seed)``, drawn in the
@@ -70,6 +71,8 @@ WORKLOADS = {
                  description="causal forward+backward with saved LSE"),
         Workload("causal1m", 1, 32, 128, 1048576, 8, 512, 1, seed=1005, std=128 ** -0.5,
                  description="million-token causal forward"),
+        Workload("causal16k", 1, 32, 128, 16384, 8, 512, 1, backward=True, seed=1006,
+                 description="profiling size: causal forward+backward, every input larger than L2"),
     ]
 }
 
