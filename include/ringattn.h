@@ -65,7 +65,8 @@ enum {
   RA_ERR_WORKSPACE = 7,      /* workspace NULL or smaller than ra_workspace_size() */
   RA_ERR_CUDA = 8,           /* a CUDA runtime call failed (launch, attribute, tensor map) */
   RA_ERR_DEVICE_TIMEOUT = 9, /* device-side bounded wait ran out (reported by ra_get_device_status) */
-  RA_ERR_ORDER = 10          /* ring_order is not a permutation of 0..ring_size-1 */
+  RA_ERR_ORDER = 10,         /* ring_order is not a permutation of 0..ring_size-1 */
+  RA_ERR_STATIC_LIMIT = 11   /* problem needs more scratch than ra_forward_static's fixed array */
 };
 
 typedef struct {
@@ -164,6 +165,29 @@ int ra_finalize(const ra_tensor* o_acc, const ra_tensor* m, const ra_tensor* l, 
  * may alias o_a / lse_a (element-wise in place). */
 int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* o_b, const ra_tensor* lse_b,
                  ra_tensor* o_out, ra_tensor* lse_out, void* stream);
+
+/* Forward that allocates nothing, for callers that cannot allocate device
+ * memory: a host program that links only this library and owns no device
+ * allocator, or code running under a fixed, pre-planned memory budget where a
+ * cudaMalloc could fail or implicitly synchronize the device.  The paper has
+ * no counterpart for this entry point: it is an addition of this library.
+ * Same arguments, semantics and results as ra_forward minus the workspace:
+ * the scratch ra_forward would take from `workspace` (per-128-token tile
+ * metadata, used only when attention_bias or segment_ids is given) lives in
+ * one file-scope device array of RA_STATIC_SCRATCH_BYTES (1 MiB), enough for
+ * B * ceil(S / 128) <= 65536 (for example B = 8 at 1M tokens).  Larger
+ * problems return RA_ERR_STATIC_LIMIT and launch nothing.
+ *  - The array is held by every GPU that loads the library until the process
+ *    exits.  The first call on a device (with that device current) looks up
+ *    the array's device address once; make that first call before any stream
+ *    capture.
+ *  - Every call shares the array and it keeps the last call's contents.  All
+ *    of it that a call reads is rewritten by that call first, so nothing has
+ *    to be cleared, but calls that overlap on the GPU (concurrent streams)
+ *    race on it: serialize them. */
+#define RA_STATIC_SCRATCH_BYTES (1u << 20)
+int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* attention_bias,
+                      const ra_tensor* segment_ids, const ra_params* p, ra_tensor* o, ra_tensor* lse, void* stream);
 
 /* Synchronizes `stream`, returns the device status word of the current
  * device (RA_OK or RA_ERR_DEVICE_TIMEOUT) and clears it.  RA_ERR_CUDA if

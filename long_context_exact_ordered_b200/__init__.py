@@ -15,12 +15,13 @@ from .api import (  # noqa: F401
     ring_step,
     ringattention,
     ringattention_backward,
+    ringattention_static,
     workspace_size,
 )
 from ._lib import RingAttnError, load  # noqa: F401
 
 __all__ = [
-    "ringattention", "ringattention_backward", "ring_step", "init_state", "finalize", "lse_merge",
+    "ringattention", "ringattention_backward", "ringattention_static", "ring_step", "init_state", "finalize", "lse_merge",
     "device_status", "count_visible_pairs", "ring_schedule", "workspace_size", "RingAttentionFunction",
     "RingAttnError", "load",
 ]

@@ -17,7 +17,7 @@ RA_MAX_RING = 64
 ERRORS = {
     0: "RA_OK", 1: "RA_ERR_NULL", 2: "RA_ERR_DTYPE", 3: "RA_ERR_SHAPE", 4: "RA_ERR_STRIDE",
     5: "RA_ERR_DIVISIBILITY", 6: "RA_ERR_UNSUPPORTED", 7: "RA_ERR_WORKSPACE", 8: "RA_ERR_CUDA",
-    9: "RA_ERR_DEVICE_TIMEOUT", 10: "RA_ERR_ORDER",
+    9: "RA_ERR_DEVICE_TIMEOUT", 10: "RA_ERR_ORDER", 11: "RA_ERR_STATIC_LIMIT",
 }
 
 
@@ -52,6 +52,7 @@ _vp = ctypes.c_void_p
 SIGNATURES = {
     "ra_workspace_size": (ctypes.c_size_t, [ctypes.c_int, _T, _P, ctypes.c_int, ctypes.c_int]),
     "ra_forward": (ctypes.c_int, [_T, _T, _T, _T, _T, _P, _T, _T, _vp, ctypes.c_size_t, _vp]),
+    "ra_forward_static": (ctypes.c_int, [_T, _T, _T, _T, _T, _P, _T, _T, _vp]),
     "ra_backward": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, _T, _T, _P, _T, _T, _T, _vp, ctypes.c_size_t, _vp]),
     "ra_step": (ctypes.c_int, [_T, _T, _T, ctypes.c_int64, ctypes.c_int64, _T, _T, _T, _P, _T, _T, _T, _vp]),
     "ra_finalize": (ctypes.c_int, [_T, _T, _T, _T, _T, _vp]),

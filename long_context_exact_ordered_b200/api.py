@@ -111,6 +111,27 @@ def ringattention(q, k, v, attention_bias=None, segment_ids=None, query_chunk_si
     return out, lse
 
 
+def ringattention_static(q, k, v, attention_bias=None, segment_ids=None, query_chunk_size=512,
+                         key_chunk_size=512, causal_block_size=None, ring_size=1, ring_order=None, out=None,
+                         lse=None):
+    """ringattention without any device allocation by the library: its scratch is a
+    fixed static device array (see ra_forward_static).  For callers that cannot
+    allocate device memory; ``out`` and ``lse`` may be preallocated so that this
+    wrapper allocates nothing either."""
+    B, S, H, D = q.shape
+    p = _params(S, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order)
+    if out is None:
+        out = torch.empty_like(q, memory_format=torch.contiguous_format)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    tq, tk, tv, to, tl = _tensor(q), _tensor(k), _tensor(v), _tensor(out), _tensor(lse)
+    tb, ts = _tensor(attention_bias), _tensor(segment_ids)
+    code = load().ra_forward_static(ctypes.byref(tq), ctypes.byref(tk), ctypes.byref(tv), _ref(tb), _ref(ts),
+                                    ctypes.byref(p), ctypes.byref(to), ctypes.byref(tl), _stream())
+    check(code, "ra_forward_static")
+    return out, lse
+
+
 def ringattention_backward(q, k, v, o, lse, do, attention_bias=None, segment_ids=None, query_chunk_size=512,
                            key_chunk_size=512, causal_block_size=None, ring_size=1, ring_order=None,
                            grad_dtype=None, workspace=None, out=None, prof_events=None):

@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <unordered_map>
 #include <vector>
 
@@ -17,6 +18,12 @@
 #include "ra_simt.cuh"
 
 using namespace ra;
+
+// Fixed scratch for ra_forward_static (tile metadata), one copy per device.
+// Host code must not pass this symbol to a kernel directly: on the host it is
+// only a stand-in, so its device address is looked up with
+// cudaGetSymbolAddress (per device, with that device current).
+static __device__ __align__(256) unsigned char g_ra_static_scratch[RA_STATIC_SCRATCH_BYTES];
 
 namespace {
 
@@ -362,6 +369,8 @@ const char* ra_strerror(int code) {
     case RA_ERR_CUDA: return "CUDA runtime error";
     case RA_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait ran out";
     case RA_ERR_ORDER: return "ring_order is not a permutation of 0..ring_size-1";
+    case RA_ERR_STATIC_LIMIT:
+      return "problem needs more scratch than ra_forward_static provides (B * ceil(S/128) must be <= 65536)";
     default: return "unknown error";
   }
 }
@@ -680,6 +689,31 @@ int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* 
               dt == RA_BF16};
   lse_merge_kernel<<<(unsigned)ceil_div64(n, 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return last_cuda();
+}
+
+int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* attention_bias,
+                      const ra_tensor* segment_ids, const ra_params* p, ra_tensor* o, ra_tensor* lse, void* stream) {
+  // Device address of the static scratch, looked up once per device.
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  if (!q || q->ndim != 4) return q ? RA_ERR_SHAPE : RA_ERR_NULL;
+  if (q->shape[0] < 0 || q->shape[1] < 0 || q->shape[2] < 0 || q->shape[3] < 0) return RA_ERR_SHAPE;
+  const bool need_meta = attention_bias || segment_ids;
+  const WsLayout w = ws_layout(0, q->shape[0], q->shape[1], q->shape[2], q->shape[3], need_meta);
+  if (w.total > RA_STATIC_SCRATCH_BYTES) return RA_ERR_STATIC_LIMIT;
+  void* scratch = nullptr;
+  if (w.total > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_ra_static_scratch) != cudaSuccess || !ptr) return RA_ERR_CUDA;
+      addr[dev] = ptr;
+    }
+    scratch = addr[dev];
+  }
+  return ra_forward(q, k, v, attention_bias, segment_ids, p, o, lse, scratch, RA_STATIC_SCRATCH_BYTES, stream);
 }
 
 int ra_get_device_status(void* stream) {

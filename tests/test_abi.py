@@ -41,7 +41,7 @@ def test_struct_layout_matches_header():
 
 def test_strerror_covers_codes():
     lib = _lib.load()
-    for code in range(0, 11):
+    for code in range(0, 12):
         s = lib.ra_strerror(code).decode()
         assert s and s != "unknown error"
     assert lib.ra_strerror(999).decode() == "unknown error"
