@@ -21,12 +21,16 @@
 // Roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 4-7 "softmax" (thread = key row: P^T, dS^T, final dK/dV epilogue),
 // warps 8-11 dQ readout (thread = head-dim lane d of dQ^T).
-// TMEM (512 columns): S^T [0,64) dP^T [64,128) dQ^T [128,192) P^T [192,224)
-// dS^T [224,256) dK [256,384) dV [384,512).
+// TMEM (512 columns): two 128-column slots, then dK [256,384), dV [384,512).
+// Query tile n uses slot n % 2: S^T -> [0,64), dP^T -> [64,128); the softmax
+// group overwrites [0,32) with P^T and [32,64) with dS^T (bf16), and dQ^T(n)
+// lands in [64,128) once dP^T has been read.  A slot is reused two tiles
+// later, after the readout group has taken dQ^T out of it.
 //
-// Overlap: S^T(i+1), dP^T(i+1) are issued as soon as the softmax group has
-// read S^T(i), dP^T(i), ahead of dV(i), dK(i), dQ^T(i), so the softmax of
-// tile i+1 runs while the tensor core finishes tile i.
+// Overlap: with two slots the "head" products of tile n+1 (S^T, dP^T) are
+// computed while the softmax group works on tile n, and the issuing thread
+// polls both "tail ready" (dV, dK, dQ^T of the oldest tile) and "head ready"
+// (slot and query stage free) so the tensor core is fed whichever is ready.
 #pragma once
 
 #include <cuda.h>
@@ -46,33 +50,33 @@ struct BwdLayout {
   static constexpr int Q_BYTES = QT * D * 2;      // 16 KB
   static constexpr int Q_CHUNK = QT * 128;        // 8 KB box: 64 rows x 128 B
   static constexpr int DS_BYTES = kTile * QT * 2; // 16 KB: 128 keys x 64 queries bf16
-  static constexpr int NS = 2;                    // query-side stages
+  static constexpr int NS = 3;                    // query-side stages (two tiles in flight + one loading)
+  static constexpr int NSLOT = 2;                 // TMEM slots
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
   static constexpr int OFF_Q = OFF_V + KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + NS * Q_BYTES;
   static constexpr int OFF_DS = OFF_DO + NS * Q_BYTES;
-  static constexpr int OFF_LD = OFF_DS + 2 * DS_BYTES;   // per stage: lse2[64], delta[64]
+  static constexpr int OFF_LD = OFF_DS + NSLOT * DS_BYTES;   // per stage: lse2[64], delta[64]
   static constexpr int LD_BYTES = 2 * QT * 4;
   static constexpr int OFF_BAR = OFF_LD + NS * LD_BYTES;
   static constexpr int B_KV = 0;
-  static constexpr int B_QF = 1;                  // [NS]
-  static constexpr int B_QE = B_QF + NS;          // [NS]
-  static constexpr int B_SFULL = B_QE + NS;
-  static constexpr int B_DPFULL = B_SFULL + 1;
-  static constexpr int B_DSREADY = B_DPFULL + 1;
-  static constexpr int B_MMADONE = B_DSREADY + 1;
-  static constexpr int B_DQFULL = B_MMADONE + 1;
-  static constexpr int B_DQFREE = B_DQFULL + 1;
-  static constexpr int B_DSBFREE = B_DQFREE + 1;  // [2]
-  static constexpr int B_FINAL = B_DSBFREE + 2;
+  static constexpr int B_QF = 1;                  // [NS] query stage loaded
+  static constexpr int B_QE = B_QF + NS;          // [NS] query stage free
+  static constexpr int B_SFULL = B_QE + NS;       // [NSLOT] S^T computed
+  static constexpr int B_DPFULL = B_SFULL + NSLOT;   // [NSLOT] dP^T computed
+  static constexpr int B_DSREADY = B_DPFULL + NSLOT; // [NSLOT] P^T, dS^T written (128 arrivals)
+  static constexpr int B_DQFULL = B_DSREADY + NSLOT; // [NSLOT] dQ^T computed
+  static constexpr int B_SLOTFREE = B_DQFULL + NSLOT;  // [NSLOT] dQ^T read out (128 arrivals)
+  static constexpr int B_FINAL = B_SLOTFREE + NSLOT;
   static constexpr int NBAR = B_FINAL + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_ST = 0, COL_DPT = 64, COL_DQT = 128, COL_PT = 192, COL_DST = 224, COL_DK = 256,
-                            COL_DV = 384;
+  static constexpr uint32_t SLOT_COLS = 128;
+  static constexpr uint32_t SLOT_ST = 0, SLOT_DPT = 64, SLOT_PT = 0, SLOT_DST = 32, SLOT_DQT = 64;
+  static constexpr uint32_t COL_DK = 256, COL_DV = 384;
   static constexpr int THREADS = 384;
 };
 
@@ -120,10 +124,11 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* gbase = smem_raw + (sbase - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // Longest units first: under causal masking the first key tiles meet the most query tiles.
-  const int BH = p.B * p.H;
-  const int kt = blockIdx.x / BH;
-  const int bh = blockIdx.x % BH;
+  // Head-major order: the resident CTAs work on the key tiles of one or two
+  // heads at a time, so that head's Q / dO stream stays in L2; within a head
+  // the first key tiles (most query tiles under causal masking) go first.
+  const int bh = blockIdx.x / p.rd.ntiles;
+  const int kt = blockIdx.x % p.rd.ntiles;
   const int b = bh / p.H, h = bh % p.H;
   const int64_t k0 = (int64_t)kt * kTile;
   const int64_t S = p.rd.S;
@@ -135,14 +140,13 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(L::B_KV), 1);
     for (int i = 0; i < L::NS; ++i) { mbar_init(bar(L::B_QF + i), 1); mbar_init(bar(L::B_QE + i), 1); }
-    mbar_init(bar(L::B_SFULL), 1);
-    mbar_init(bar(L::B_DPFULL), 1);
-    mbar_init(bar(L::B_DSREADY), 128);
-    mbar_init(bar(L::B_MMADONE), 1);
-    mbar_init(bar(L::B_DQFULL), 1);
-    mbar_init(bar(L::B_DQFREE), 128);
-    mbar_init(bar(L::B_DSBFREE + 0), 1);
-    mbar_init(bar(L::B_DSBFREE + 1), 1);
+    for (int i = 0; i < L::NSLOT; ++i) {
+      mbar_init(bar(L::B_SFULL + i), 1);
+      mbar_init(bar(L::B_DPFULL + i), 1);
+      mbar_init(bar(L::B_DSREADY + i), 128);
+      mbar_init(bar(L::B_DQFULL + i), 1);
+      mbar_init(bar(L::B_SLOTFREE + i), 128);
+    }
     mbar_init(bar(L::B_FINAL), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -200,7 +204,7 @@ __global__ void __launch_bounds__(384, 1)
         if (i >= 0) ra_wait_drain(bar(L::B_QF + i % L::NS), (i / L::NS) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (event loop)
     if (lane == 0) {
       constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, L::QT, false, false);
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);
@@ -221,53 +225,61 @@ __global__ void __launch_bounds__(384, 1)
           mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_base + kk * 2048, L::Q_CHUNK, 1024), IDESC_KV,
                  (acc || kk > 0) ? 1u : 0u);
       };
-      auto issue_dq = [&](uint32_t ds_base) {
+      auto issue_dq = [&](uint32_t d_tmem, uint32_t ds_base) {
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ss(tmem + L::COL_DQT, smem_desc_sw128(ka + kk * 2048, L::KV_CHUNK, 1024),
+          mma_ss(d_tmem, smem_desc_sw128(ka + kk * 2048, L::KV_CHUNK, 1024),
                  smem_desc_sw128(ds_base + kk * 2048, L::DS_BYTES, 1024), IDESC_DQ, kk > 0);
       };
-      bool ok = ra_wait(bar(L::B_KV), 0, abort_flag);
-      if (ok && !dead) {
+      // number of query tiles this key tile visits
+      int N = 0;
+      if (!dead) {
         QIter it;
         q_iter_init(it, p.rd, k0, meta_b, use_seg);
-        int32_t q = q_iter_next(it, p.rd);
-        if (q >= 0) {
-          ok = ra_wait(bar(L::B_QF + 0), 0, abort_flag);
-          if (ok) {
+        while (q_iter_next(it, p.rd) >= 0) ++N;
+      }
+      bool ok = ra_wait(bar(L::B_KV), 0, abort_flag);
+      int hd = 0, tl = 0;    // next head (S^T, dP^T) and next tail (dV, dK, dQ^T) to issue
+      long long idle_since = clock64();
+      while (ok && tl < N) {
+        bool progress = false;
+        if (tl < hd) {
+          const int s = tl & 1;
+          if (mbar_probe(bar(L::B_DSREADY + s), (tl >> 1) & 1)) {
             tc_fence_after();
-            issue_sd(tmem + L::COL_ST, ka, sbase + L::OFF_Q);
-            mma_commit(bar(L::B_SFULL));
-            issue_sd(tmem + L::COL_DPT, va, sbase + L::OFF_DO);
-            mma_commit(bar(L::B_DPFULL));
-          }
-          for (int n = 0; ok; ++n) {
-            const int32_t qn = q_iter_next(it, p.rd);
-            const bool last = qn < 0;
-            const int st = n % L::NS, st1 = (n + 1) % L::NS;
-            if (!(ok = ra_wait(bar(L::B_DSREADY), n & 1, abort_flag))) break;
-            tc_fence_after();
-            if (!last) {
-              if (!(ok = ra_wait(bar(L::B_QF + st1), ((n + 1) / L::NS) & 1, abort_flag))) break;
-              tc_fence_after();
-              issue_sd(tmem + L::COL_ST, ka, sbase + L::OFF_Q + st1 * L::Q_BYTES);
-              mma_commit(bar(L::B_SFULL));
-              issue_sd(tmem + L::COL_DPT, va, sbase + L::OFF_DO + st1 * L::Q_BYTES);
-              mma_commit(bar(L::B_DPFULL));
-            }
-            issue_kv(tmem + L::COL_DV, tmem + L::COL_PT, sbase + L::OFF_DO + st * L::Q_BYTES, n > 0);
-            issue_kv(tmem + L::COL_DK, tmem + L::COL_DST, sbase + L::OFF_Q + st * L::Q_BYTES, n > 0);
-            mma_commit(bar(L::B_MMADONE));
-            if (n > 0) {
-              if (!(ok = ra_wait(bar(L::B_DQFREE), (n - 1) & 1, abort_flag))) break;
-              tc_fence_after();
-            }
-            issue_dq(sbase + L::OFF_DS + (n & 1) * L::DS_BYTES);
-            mma_commit(bar(L::B_DQFULL));
-            mma_commit(bar(L::B_DSBFREE + (n & 1)));
+            const uint32_t slot = tmem + s * L::SLOT_COLS;
+            const int st = tl % L::NS;
+            issue_kv(tmem + L::COL_DV, slot + L::SLOT_PT, sbase + L::OFF_DO + st * L::Q_BYTES, tl > 0);
+            issue_kv(tmem + L::COL_DK, slot + L::SLOT_DST, sbase + L::OFF_Q + st * L::Q_BYTES, tl > 0);
+            issue_dq(slot + L::SLOT_DQT, sbase + L::OFF_DS + s * L::DS_BYTES);
+            mma_commit(bar(L::B_DQFULL + s));
             mma_commit(bar(L::B_QE + st));
-            if (last) break;
+            ++tl;
+            progress = true;
           }
+        }
+        if (hd < N && hd < tl + L::NSLOT) {
+          const int s = hd & 1, st = hd % L::NS;
+          const bool slot_free = hd < L::NSLOT || mbar_probe(bar(L::B_SLOTFREE + s), ((hd >> 1) - 1) & 1);
+          if (slot_free && mbar_probe(bar(L::B_QF + st), (hd / L::NS) & 1)) {
+            tc_fence_after();
+            const uint32_t slot = tmem + s * L::SLOT_COLS;
+            issue_sd(slot + L::SLOT_ST, ka, sbase + L::OFF_Q + st * L::Q_BYTES);
+            mma_commit(bar(L::B_SFULL + s));
+            issue_sd(slot + L::SLOT_DPT, va, sbase + L::OFF_DO + st * L::Q_BYTES);
+            mma_commit(bar(L::B_DPFULL + s));
+            ++hd;
+            progress = true;
+          }
+        }
+        if (progress) {
+          idle_since = clock64();
+        } else if (*abort_flag) {
+          ok = false;
+        } else if (clock64() - idle_since > RA_SPIN_BUDGET) {
+          raise_status(9 /* RA_ERR_DEVICE_TIMEOUT */);
+          *abort_flag = 1;
+          ok = false;
         }
       }
       mma_commit(bar(L::B_FINAL));
@@ -294,14 +306,15 @@ __global__ void __launch_bounds__(384, 1)
       QIter it;
       q_iter_init(it, p.rd, k0, meta_b, use_seg);
       for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
-        const int st = n % L::NS;
+        const int st = n % L::NS, s = n & 1;
+        const uint32_t slot = trow + s * L::SLOT_COLS;
         const int64_t q0 = (int64_t)q * L::QT;
         if (!(ok = ra_wait_warp(bar(L::B_QF + st), (n / L::NS) & 1, abort_flag))) break;
-        if (!(ok = ra_wait_warp(bar(L::B_SFULL), n & 1, abort_flag))) break;
+        if (!(ok = ra_wait_warp(bar(L::B_SFULL + s), (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         uint32_t sr[64];
-        tmem_ld32(trow + L::COL_ST, sr);
-        tmem_ld32(trow + L::COL_ST + 32, sr + 32);
+        tmem_ld32(slot + L::SLOT_ST, sr);
+        tmem_ld32(slot + L::SLOT_ST + 32, sr + 32);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 64; ++c) reg_fence(sr[c]);
@@ -347,11 +360,11 @@ __global__ void __launch_bounds__(384, 1)
         float pr[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) pr[c] = ex2_approx(x[c]);
-        if (!(ok = ra_wait_warp(bar(L::B_DPFULL), n & 1, abort_flag))) break;
+        if (!(ok = ra_wait_warp(bar(L::B_DPFULL + s), (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         uint32_t dr[64];
-        tmem_ld32(trow + L::COL_DPT, dr);
-        tmem_ld32(trow + L::COL_DPT + 32, dr + 32);
+        tmem_ld32(slot + L::SLOT_DPT, dr);
+        tmem_ld32(slot + L::SLOT_DPT + 32, dr + 32);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 64; ++c) reg_fence(dr[c]);
@@ -363,23 +376,19 @@ __global__ void __launch_bounds__(384, 1)
           pp[c >> 1] = pack_bf16x2(pr[c], pr[c + 1]);
           dd[c >> 1] = pack_bf16x2(ds0, ds1);
         }
-        // P^T / dS^T columns of TMEM are free once dV(n-1), dK(n-1) completed
-        if (n > 0 && !(ok = ra_wait_warp(bar(L::B_MMADONE), (n - 1) & 1, abort_flag))) break;
-        tc_fence_after();
-        tmem_st32(trow + L::COL_PT, pp);
-        tmem_st32(trow + L::COL_DST, dd);
+        // P^T and dS^T into this slot (its S^T / first half was read above).
+        tmem_st32(slot + L::SLOT_PT, pp);
+        tmem_st32(slot + L::SLOT_DST, dd);
         // dS^T into shared memory for dQ^T = K^T dS^T (MN-major, 128-byte swizzle):
         // key row `row` is one 128-byte line; 16-byte chunk c lands at c ^ (row % 8).
-        const int buf = n & 1;
-        if (n >= 2 && !(ok = ra_wait_warp(bar(L::B_DSBFREE + buf), ((n >> 1) - 1) & 1, abort_flag))) break;
-        const uint32_t line = sbase + L::OFF_DS + buf * L::DS_BYTES + row * 128;
+        const uint32_t line = sbase + L::OFF_DS + s * L::DS_BYTES + row * 128;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
           st_shared_v4(line + ((c ^ (row & 7)) << 4), dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::B_DSREADY));
+        mbar_arrive(bar(L::B_DSREADY + s));
       }
     }
     // ---------------------------------------------------------- dK / dV epilogue
@@ -433,22 +442,23 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------ dQ readout: thread = head-dim lane d
     const int sub = warp & 3;
     const int d = sub * 32 + lane;
-    const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16) + L::COL_DQT;
+    const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
     if (!dead) {
       QIter it;
       q_iter_init(it, p.rd, k0, meta_b, use_seg);
       int n = 0;
       for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
-        if (!ra_wait_warp(bar(L::B_DQFULL), n & 1, abort_flag)) break;
+        const int s = n & 1;
+        if (!ra_wait_warp(bar(L::B_DQFULL + s), (n >> 1) & 1, abort_flag)) break;
         tc_fence_after();
         uint32_t r[64];
-        tmem_ld32(trow, r);
-        tmem_ld32(trow + 32, r + 32);
+        tmem_ld32(trow + s * L::SLOT_COLS + L::SLOT_DQT, r);
+        tmem_ld32(trow + s * L::SLOT_COLS + L::SLOT_DQT + 32, r + 32);
         tmem_ld_wait();
 #pragma unroll
         for (int c = 0; c < 64; ++c) reg_fence(r[c]);
         tc_fence_before();
-        mbar_arrive(bar(L::B_DQFREE));
+        mbar_arrive(bar(L::B_SLOTFREE + s));
         const int64_t q0 = (int64_t)q * L::QT;
         float* dst = p.dqacc + ((int64_t)bh * S + q0) * D + d;
         const int64_t nvalid = S - q0;

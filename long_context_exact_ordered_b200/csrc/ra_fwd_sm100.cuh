@@ -26,10 +26,11 @@
 // 8 (log2 units), so unnormalised probabilities stay <= 2^8 and the final
 // O / l is unchanged.
 //
-// Pipeline: S_q(t+1) reuses the TMEM columns holding P_q(t), so the issuer
-// waits for PV_q(t) to complete before issuing S_q(t+1).  Order per tile:
-// PV0(t), S0(t+1), PV1(t), S1(t+1): while softmax 1 works on S1(t) the
-// tensor core runs PV0/S0, and vice versa.
+// Pipeline: order per key tile PV0(t), S0(t+1), PV1(t), S1(t+1): while
+// softmax 1 works on S1(t) the tensor core runs PV0/S0, and vice versa.
+// S_q(t+1) reuses the TMEM columns holding P_q(t); it is issued by the same
+// thread right behind PV_q(t) and the tensor pipe executes a thread's MMAs
+// in issue order.
 #pragma once
 
 #include <cuda.h>
@@ -105,11 +106,11 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t* gbase = smem_raw + (sbase - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // LPT order: the longest causal units (last query pairs) launch first.
-  const int BH = p.B * p.H;
+  // Head-major order (resident CTAs share one head's K / V in L2); within a
+  // head the longest causal units (last query pairs) launch first.
   const int unit = blockIdx.x;
-  const int pair = p.npairs - 1 - unit / BH;
-  const int bh = unit % BH;
+  const int pair = p.npairs - 1 - unit % p.npairs;
+  const int bh = unit / p.npairs;
   const int b = bh / p.H, h = bh % p.H;
   const int64_t q0 = (int64_t)pair * 2 * kTile;
   const int64_t S = p.rd.S;
@@ -232,9 +233,10 @@ __global__ void __launch_bounds__(384, 1)
           issue_pv(0, vs, n > 0);
           mma_commit(bar(L::B_PVDONE + 0));
           if (!last) {
+            // S0(n+1) overwrites the TMEM columns PV0(n) reads P0 from; the
+            // tensor pipe executes this thread's MMAs in issue order, so it is
+            // issued right behind PV0(n) without waiting for its completion.
             if (!(ok = ra_wait(bar(L::B_KFULL + ks1), ((n + 1) / L::KS) & 1, abort_flag))) break;
-            if (!(ok = ra_wait(bar(L::B_PVDONE + 0), ph, abort_flag))) break;
-            tc_fence_after();
             issue_s(0, ks1);
             mma_commit(bar(L::B_SFULL + 0));
           }
@@ -245,8 +247,6 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit(bar(L::B_PVDONE + 1));
           mma_commit(bar(L::B_VEMPTY + vs));
           if (!last) {
-            if (!(ok = ra_wait(bar(L::B_PVDONE + 1), ph, abort_flag))) break;
-            tc_fence_after();
             issue_s(1, ks1);
             mma_commit(bar(L::B_SFULL + 1));
             mma_commit(bar(L::B_KEMPTY + ks1));
@@ -299,9 +299,11 @@ __global__ void __launch_bounds__(384, 1)
 
       const int64_t k0 = (int64_t)t * kTile;
       const int4 km = meta_b ? load_meta(meta_b + t) : make_int4(0, 0, 3, 0);
-      // scale (+ bias); loads are issued 32 keys at a time (the empty asm keeps
-      // the compiler from hoisting all 128 and spilling)
-      if (use_bias && !(km.z & kMetaAllZero)) {
+      // Scores stay raw (the scale is folded into the exponent's FMA) unless a
+      // non-zero bias must be added first; loads are issued 32 keys at a time
+      // (the empty asm keeps the compiler from hoisting all 128 and spilling).
+      const bool has_bias = use_bias && !(km.z & kMetaAllZero);
+      if (has_bias) {
         const float* bp = p.bias + b * p.bias_sb;
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
@@ -312,9 +314,6 @@ __global__ void __launch_bounds__(384, 1)
           }
           asm volatile("" ::: "memory");
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] *= p.scale_log2;
       }
       // per-element mask on diagonal / ragged / mixed-segment tiles
       if (tile_needs_mask(p.rd, q_first, t, use_seg, qm, km)) {
@@ -342,16 +341,15 @@ __global__ void __launch_bounds__(384, 1)
           x[c] = vis ? x[c] : -INFINITY;
         }
       }
-      // tile max
-      float mx0 = x[0], mx1 = x[1], mx2 = x[2], mx3 = x[3];
+      // tile max (three-input max, two independent chains)
+      float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
 #pragma unroll
       for (int c = 4; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, x[c]);
-        mx1 = fmaxf(mx1, x[c + 1]);
-        mx2 = fmaxf(mx2, x[c + 2]);
-        mx3 = fmaxf(mx3, x[c + 3]);
+        mx0 = fmax3(mx0, x[c], x[c + 1]);
+        mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      const float sc = has_bias ? 1.f : p.scale_log2;   // x * sc is the score in log2 units
+      const float mx = fmaxf(mx0, mx1) * sc;
       const bool need = mx > m_ref + kRescaleThreshold;
       float alpha = 1.f;
       if (need) {
@@ -361,7 +359,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (n > 0 && __any_sync(0xffffffffu, need)) {
         // rescale this warp's O rows in TMEM (PV of the previous tile has completed:
-        // S_q(n) was issued only after it)
+        // the commit that released S_q(n) covers it)
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t orow[32];
@@ -375,22 +373,26 @@ __global__ void __launch_bounds__(384, 1)
           tmem_st32(tO_row + c, orow);
         }
       }
-      const float ref = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float l0 = 0.f, l1 = 0.f;
+      const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float e0 = ex2_approx(x[half * 64 + c] - ref);
-          const float e1 = ex2_approx(x[half * 64 + c + 1] - ref);
-          l0 += e0;
-          l1 += e1;
+        for (int c = 0; c < 64; c += 4) {
+          const int i = half * 64 + c;
+          float a0, a1, a2, a3;
+          ffma2(a0, a1, x[i], x[i + 1], sc, sc, nref, nref);
+          ffma2(a2, a3, x[i + 2], x[i + 3], sc, sc, nref, nref);
+          const float e0 = ex2_approx(a0), e1 = ex2_approx(a1), e2 = ex2_approx(a2), e3 = ex2_approx(a3);
+          fadd2(l0, l1, l0, l1, e0, e1);
+          fadd2(l2, l3, l2, l3, e2, e3);
           pk[c >> 1] = pack_bf16x2(e0, e1);
+          pk[(c >> 1) + 1] = pack_bf16x2(e2, e3);
         }
         tmem_st32(tS_row + half * 32, pk);
       }
-      l += l0 + l1;
+      l += (l0 + l1) + (l2 + l3);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::B_PFULL + qt));
