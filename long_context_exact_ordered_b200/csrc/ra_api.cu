@@ -187,6 +187,20 @@ int make_tmap_bshd(CUtensorMap* m, const ra_tensor* t, int rows) {
 
 int last_cuda() { return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA; }
 
+// fp32 [BH][S][D] workspace -> 3-D map (D, S, BH), box D x rows x 1, no swizzle.
+int make_tmap_dqacc(CUtensorMap* m, float* base, int64_t BH, int64_t S, int64_t D, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return RA_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)S * D * 4};
+  cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? RA_OK : RA_ERR_CUDA;
+}
+
 // Profiling hooks of ra_params: events recorded around the main kernel.
 struct ProfScope {
   cudaEvent_t b = nullptr, e = nullptr;
@@ -301,11 +315,13 @@ int launch_bwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v,
                      const MaskArgs& mk, const RingDesc& rd, const int4* meta, const WsLayout& w, char* ws,
                      ra_tensor* dk, ra_tensor* dv, cudaStream_t st) {
   using L = BwdLayout;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   RA_TRY(make_tmap_bshd(&tq, q, L::QT));
   RA_TRY(make_tmap_bshd(&tk, k, kTile));
   RA_TRY(make_tmap_bshd(&tv, v, kTile));
   RA_TRY(make_tmap_bshd(&tdo, d_o, L::QT));
+  RA_TRY(make_tmap_dqacc(&tdq, reinterpret_cast<float*>(ws + w.dqacc), q->shape[0] * q->shape[2], q->shape[1],
+                         L::D, L::QT));
   BwdParams prm;
   std::memset(&prm, 0, sizeof(prm));
   prm.rd = rd;
@@ -338,7 +354,7 @@ int launch_bwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v,
   if (cudaFuncSetAttribute(ra_bwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
       cudaSuccess)
     return RA_ERR_CUDA;
-  ra_bwd_sm100_kernel<<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, prm);
+  ra_bwd_sm100_kernel<<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, tdq, prm);
   return last_cuda();
 }
 

@@ -15,8 +15,9 @@
 //   dV  += P^T dO_i             (TS: P^T bf16 in TMEM, dO MN-major)
 //   dK  += dS^T Q_i             (TS: dS^T bf16 in TMEM, Q MN-major)
 //   dQ^T = K^T dS^T             (SS: K and dS^T both MN-major) -> TMEM [128 x 64]
-// dQ^T is read back by a dedicated warpgroup and reduced into an fp32
-// workspace (atomic adds; dQ gathers contributions from every key tile).
+// dQ^T is read back by a dedicated warpgroup, staged in shared memory as a
+// [64 queries x D] fp32 tile and added into the fp32 dQ workspace with one
+// TMA bulk reduce-add per tile (dQ gathers contributions from every key tile).
 //
 // Roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
 // warps 4-7 "softmax" (thread = key row: P^T, dS^T, final dK/dV epilogue),
@@ -59,7 +60,9 @@ struct BwdLayout {
   static constexpr int OFF_DS = OFF_DO + NS * Q_BYTES;
   static constexpr int OFF_LD = OFF_DS + NSLOT * DS_BYTES;   // per stage: lse2[64], delta[64]
   static constexpr int LD_BYTES = 2 * QT * 4;
-  static constexpr int OFF_BAR = OFF_LD + NS * LD_BYTES;
+  static constexpr int OFF_DQS = OFF_LD + NS * LD_BYTES;    // dQ staging [64][D] fp32
+  static constexpr int DQS_BYTES = QT * D * 4;               // 32 KB
+  static constexpr int OFF_BAR = OFF_DQS + DQS_BYTES;
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1;                  // [NS] query stage loaded
   static constexpr int B_QE = B_QF + NS;          // [NS] query stage free
@@ -69,7 +72,9 @@ struct BwdLayout {
   static constexpr int B_DQFULL = B_DSREADY + NSLOT; // [NSLOT] dQ^T computed
   static constexpr int B_SLOTFREE = B_DQFULL + NSLOT;  // [NSLOT] dQ^T read out (128 arrivals)
   static constexpr int B_FINAL = B_SLOTFREE + NSLOT;
-  static constexpr int NBAR = B_FINAL + 1;
+  static constexpr int B_DQSFULL = B_FINAL + 1;      // staging written (128 arrivals)
+  static constexpr int B_DQSFREE = B_DQSFULL + 1;    // staging read by the bulk reduce
+  static constexpr int NBAR = B_DQSFREE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
@@ -78,6 +83,8 @@ struct BwdLayout {
   static constexpr uint32_t SLOT_ST = 0, SLOT_DPT = 64, SLOT_PT = 0, SLOT_DST = 32, SLOT_DQT = 64;
   static constexpr uint32_t COL_DK = 256, COL_DV = 384;
   static constexpr int THREADS = 384;
+  static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+  static_assert(OFF_DQS % 128 == 0, "bulk reduce source alignment");
 };
 
 struct BwdParams {
@@ -101,6 +108,23 @@ struct BwdParams {
   const int4* meta;
 };
 
+// Tensor bulk reduce-add shared -> global (3-D tile, fp32 add), tracked by a bulk group.
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 // 1-D bulk copy global -> shared (16-byte aligned, size multiple of 16).
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -115,7 +139,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 __global__ void __launch_bounds__(384, 1)
     ra_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                        const __grid_constant__ BwdParams p) {
+                        const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ BwdParams p) {
   using L = BwdLayout;
   constexpr int D = L::D;
   extern __shared__ uint8_t smem_raw[];
@@ -148,6 +172,8 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(L::B_SLOTFREE + i), 128);
     }
     mbar_init(bar(L::B_FINAL), 1);
+    mbar_init(bar(L::B_DQSFULL), 128);
+    mbar_init(bar(L::B_DQSFREE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -300,6 +326,9 @@ __global__ void __launch_bounds__(384, 1)
     if (use_bias) brow = p.bias[b * p.bias_sb + jc * p.bias_ss] * kLog2e;
     const int32_t cbs = p.rd.cbs;
     const int64_t i_first = cbs > 0 ? (j / cbs) * (int64_t)cbs : 0;   // first query that can see key j
+    // A query tile starting at q0 needs the causal mask iff q0 is before the
+    // causal block of the tile's last key (no per-tile division).
+    const int64_t k_last_blk = cbs > 0 ? ((k0 + kTile - 1) / cbs) * (int64_t)cbs : 0;
     int n = 0;
     bool ok = true;
     if (!dead) {
@@ -325,7 +354,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 64; ++c) x[c] = fmaf(x[c], p.scale_log2, brow - lse2[c]);
         // per-element mask on causal-diagonal / ragged / mixed-segment tiles
         const int4 qm = meta_b ? load_meta(meta_b + q0 / kTile) : make_int4(0, 0, 3, 0);
-        const bool need_causal = cbs > 0 && (q0 / cbs) < ((k0 + kTile - 1) / cbs);
+        const bool need_causal = cbs > 0 && q0 < k_last_blk;
         const bool need_ragged = (q0 + L::QT > S) || (k0 + kTile > S);
         const bool need_seg = use_seg && !(qm.x == qm.y && km.x == km.y && qm.x == km.x);
         if (need_causal || need_ragged || need_seg || !row_valid) {
@@ -442,8 +471,12 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------ dQ readout: thread = head-dim lane d
     const int sub = warp & 3;
     const int d = sub * 32 + lane;
+    const bool leader = threadIdx.x == 256;
     const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
+    const uint32_t dqs = sbase + L::OFF_DQS;
+    bool pending = false;   // leader: a bulk reduce may still be reading the staging tile
     if (!dead) {
+      if (leader) prefetch_tmap(&tm_dq);
       QIter it;
       q_iter_init(it, p.rd, k0, meta_b, use_seg);
       int n = 0;
@@ -459,14 +492,24 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 64; ++c) reg_fence(r[c]);
         tc_fence_before();
         mbar_arrive(bar(L::B_SLOTFREE + s));
-        const int64_t q0 = (int64_t)q * L::QT;
-        float* dst = p.dqacc + ((int64_t)bh * S + q0) * D + d;
-        const int64_t nvalid = S - q0;
+        // staging tile [query c][d]: a warp writes 32 consecutive floats per row
+        if (n > 0 && !ra_wait_warp(bar(L::B_DQSFREE), (n - 1) & 1, abort_flag)) break;
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c < nvalid) atomicAdd(dst + (int64_t)c * D, __uint_as_float(r[c]) * p.scale);
+        for (int c = 0; c < 64; ++c) st_shared_f32(dqs + c * (D * 4) + d * 4, __uint_as_float(r[c]) * p.scale);
+        fence_proxy_async_smem();
+        mbar_arrive(bar(L::B_DQSFULL));
+        if (leader) {
+          if (!ra_wait(bar(L::B_DQSFULL), n & 1, abort_flag)) break;
+          // rows past S fall outside the tensor map and are not written
+          tma_reduce_add_3d(&tm_dq, dqs, 0, q * L::QT, bh);
+          bulk_commit_group();
+          pending = true;
+          bulk_wait_group_read0();
+          mbar_arrive(bar(L::B_DQSFREE));
+        }
       }
     }
+    if (leader && pending) bulk_wait_group0();
   }
 
   // ------------------------------------------------------------ teardown

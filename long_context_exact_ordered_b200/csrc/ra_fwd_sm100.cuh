@@ -73,7 +73,7 @@ struct FwdLayout {
   // registers to the two softmax warpgroups.  The host checks
   // 128*REGS_LOW + 256*REGS_HIGH <= 384 * (registers per thread at launch)
   // before launching, so the increase can always be satisfied.
-  static constexpr int REGS_LOW = 64, REGS_HIGH = 208;
+  static constexpr int REGS_LOW = 88, REGS_HIGH = 200;
   static constexpr int THREADS = 384;
 };
 
@@ -278,6 +278,11 @@ __global__ void __launch_bounds__(384, 1)
     const int4 qm = (meta_b && q_tile_idx < p.rd.ntiles) ? load_meta(meta_b + q_tile_idx) : make_int4(0, 0, 3, 0);
     const int32_t cbs = p.rd.cbs;
     const int64_t causal_jmax = cbs > 0 ? (qrow / cbs + 1) * (int64_t)cbs - 1 : S - 1;
+    // Per-tile mask test without divisions: a KV tile needs the per-element
+    // mask iff it reaches past the causal block of the tile's first query
+    // (k_last > q_blk_end), runs past S, or mixes segment ids.
+    const int64_t q_blk_end = cbs > 0 ? (q_first / cbs + 1) * (int64_t)cbs - 1 : INT64_MAX;
+    const bool q_seg_uniform = qm.x == qm.y;
 
     KvIter it;
     kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
@@ -316,7 +321,10 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
       // per-element mask on diagonal / ragged / mixed-segment tiles
-      if (tile_needs_mask(p.rd, q_first, t, use_seg, qm, km)) {
+      const int64_t k_last = k0 + kTile - 1;
+      const bool need_mask = k_last > S - 1 || k_last > q_blk_end ||
+                             (use_seg && !(q_seg_uniform && km.x == km.y && qm.x == km.x));
+      if (need_mask) {
         int64_t jmax = causal_jmax < S - 1 ? causal_jmax : S - 1;
         const int64_t lim64 = jmax - k0;
         const int lim = lim64 < -1 ? -1 : (lim64 > 127 ? 127 : (int)lim64);
