@@ -194,6 +194,15 @@ int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v
  * the synchronization itself failed. */
 int ra_get_device_status(void* stream);
 
+/* Failure-path self-test: launches one warp that waits, through the same
+ * bounded mbarrier wait the attention kernels use, on a barrier phase that
+ * nothing ever completes.  After budget_cycles clock cycles (1e3 .. 1e9) the
+ * wait gives up, records RA_ERR_DEVICE_TIMEOUT in the device status word and
+ * the kernel returns normally; read the result with ra_get_device_status().
+ * No fault, trap or hang is involved: the device context stays usable.
+ * Returns RA_ERR_UNSUPPORTED for a budget outside the range. */
+int ra_selftest_timeout(int64_t budget_cycles, void* stream);
+
 /* Static description of an error code (never NULL). */
 const char* ra_strerror(int code);
 

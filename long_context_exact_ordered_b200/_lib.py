@@ -58,6 +58,7 @@ SIGNATURES = {
     "ra_finalize": (ctypes.c_int, [_T, _T, _T, _T, _T, _vp]),
     "ra_lse_merge": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, _vp]),
     "ra_get_device_status": (ctypes.c_int, [_vp]),
+    "ra_selftest_timeout": (ctypes.c_int, [ctypes.c_int64, _vp]),
     "ra_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "ra_count_visible_pairs": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                                  ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_float)]),

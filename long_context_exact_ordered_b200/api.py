@@ -215,6 +215,13 @@ def device_status(stream=None) -> int:
     return load().ra_get_device_status(s)
 
 
+def selftest_timeout(budget_cycles: int = 2_000_000) -> int:
+    """Run the bounded-wait failure path on the device and return the status it
+    left (RA_ERR_DEVICE_TIMEOUT = 9 when the mechanism works)."""
+    check(load().ra_selftest_timeout(int(budget_cycles), _stream()), "ra_selftest_timeout")
+    return device_status()
+
+
 def _host_i32(x):
     if x is None:
         return None, None

@@ -68,20 +68,24 @@ __device__ int g_ra_status;
 __device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_ra_status, 0, code); }
 
 // Bounded wait for completion of phase `parity` of barrier `bar`.  Returns
-// false (and raises the block's abort flag) on timeout or if another role
-// already aborted.
-__device__ __forceinline__ bool ra_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+// false (and raises the block's abort flag) after `budget` clock cycles or
+// if another role already aborted.
+__device__ __forceinline__ bool ra_wait_budget(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               long long budget) {
   if (mbar_test(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_test(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > RA_SPIN_BUDGET) {
+    if (clock64() - t0 > budget) {
       raise_status(9 /* RA_ERR_DEVICE_TIMEOUT */);
       *abort_flag = 1;
       return false;
     }
   }
+}
+__device__ __forceinline__ bool ra_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+  return ra_wait_budget(bar, parity, abort_flag, RA_SPIN_BUDGET);
 }
 
 // ra_wait for every lane of a warp, with a warp-uniform result: if any lane
@@ -279,6 +283,13 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
       "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
       "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }

@@ -24,6 +24,8 @@ using namespace ra;
 // only a stand-in, so its device address is looked up with
 // cudaGetSymbolAddress (per device, with that device current).
 static __device__ __align__(256) unsigned char g_ra_static_scratch[RA_STATIC_SCRATCH_BYTES];
+// Written only by the failure-path self-test kernel (1 = its wait gave up).
+static __device__ int g_ra_selftest_result;
 
 namespace {
 
@@ -730,6 +732,14 @@ int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v
     scratch = addr[dev];
   }
   return ra_forward(q, k, v, attention_bias, segment_ids, p, o, lse, scratch, RA_STATIC_SCRATCH_BYTES, stream);
+}
+
+int ra_selftest_timeout(int64_t budget_cycles, void* stream) {
+  if (budget_cycles < 1000 || budget_cycles > 1000000000ll) return RA_ERR_UNSUPPORTED;
+  int* ptr = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_ra_selftest_result) != cudaSuccess) return RA_ERR_CUDA;
+  selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_cycles, ptr);
+  return last_cuda();
 }
 
 int ra_get_device_status(void* stream) {

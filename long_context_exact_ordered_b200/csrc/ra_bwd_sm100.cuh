@@ -19,9 +19,10 @@
 // [64 queries x D] fp32 tile and added into the fp32 dQ workspace with one
 // TMA bulk reduce-add per tile (dQ gathers contributions from every key tile).
 //
-// Roles (384 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
-// warps 4-7 "softmax" (thread = key row: P^T, dS^T, final dK/dV epilogue),
-// warps 8-11 dQ readout (thread = head-dim lane d of dQ^T).
+// Roles (512 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
+// warps 4-7 and 12-15 "softmax" (thread = key row; the two warpgroups take
+// query columns 0-31 and 32-63 of each tile: P^T, dS^T, then dK resp. dV in
+// the epilogue), warps 8-11 dQ readout (thread = head-dim lane d of dQ^T).
 // TMEM (512 columns): two 128-column slots, then dK [256,384), dV [384,512).
 // Query tile n uses slot n % 2: S^T -> [0,64), dP^T -> [64,128); the softmax
 // group overwrites [0,32) with P^T and [32,64) with dS^T (bf16), and dQ^T(n)
@@ -68,7 +69,7 @@ struct BwdLayout {
   static constexpr int B_QE = B_QF + NS;          // [NS] query stage free
   static constexpr int B_SFULL = B_QE + NS;       // [NSLOT] S^T computed
   static constexpr int B_DPFULL = B_SFULL + NSLOT;   // [NSLOT] dP^T computed
-  static constexpr int B_DSREADY = B_DPFULL + NSLOT; // [NSLOT] P^T, dS^T written (128 arrivals)
+  static constexpr int B_DSREADY = B_DPFULL + NSLOT; // [NSLOT] P^T, dS^T written (256 arrivals)
   static constexpr int B_DQFULL = B_DSREADY + NSLOT; // [NSLOT] dQ^T computed
   static constexpr int B_SLOTFREE = B_DQFULL + NSLOT;  // [NSLOT] dQ^T read out (128 arrivals)
   static constexpr int B_FINAL = B_SLOTFREE + NSLOT;
@@ -82,7 +83,7 @@ struct BwdLayout {
   static constexpr uint32_t SLOT_COLS = 128;
   static constexpr uint32_t SLOT_ST = 0, SLOT_DPT = 64, SLOT_PT = 0, SLOT_DST = 32, SLOT_DQT = 64;
   static constexpr uint32_t COL_DK = 256, COL_DV = 384;
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 512;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(OFF_DQS % 128 == 0, "bulk reduce source alignment");
 };
@@ -92,8 +93,8 @@ struct BwdParams {
   int32_t B, H;
   float scale_log2;          // log2(e) / sqrt(D)
   float scale;               // 1 / sqrt(D)
-  const float* lse2;         // [B*H][s_pad]: lse * log2(e), +inf for rows with no visible key
-  const float* delta;        // [B*H][s_pad]: <dO_i, O_i>
+  const float* lse2;         // [B*H][s_pad]: -lse * log2(e), -inf for rows with no visible key
+  const float* delta;        // [B*H][s_pad]: -<dO_i, O_i>
   int64_t s_pad;
   float* dqacc;              // [B*H][S][D] fp32, pre-zeroed
   void* dk;
@@ -136,7 +137,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     ra_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ BwdParams p) {
@@ -167,7 +168,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < L::NSLOT; ++i) {
       mbar_init(bar(L::B_SFULL + i), 1);
       mbar_init(bar(L::B_DPFULL + i), 1);
-      mbar_init(bar(L::B_DSREADY + i), 128);
+      mbar_init(bar(L::B_DSREADY + i), 256);
       mbar_init(bar(L::B_DQFULL + i), 1);
       mbar_init(bar(L::B_SLOTFREE + i), 128);
     }
@@ -312,8 +313,10 @@ __global__ void __launch_bounds__(384, 1)
       ra_wait_drain(bar(L::B_FINAL), 0);
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ softmax group: one key row per thread
+  } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+    // ------------------------------------------------------------ softmax groups: one key row per thread
+    const int half = warp >= 12;                     // query columns [32*half, 32*half + 32) of each tile
+    const int c0 = half * 32;
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
     const int64_t j = k0 + row;                      // this thread's key
@@ -329,6 +332,7 @@ __global__ void __launch_bounds__(384, 1)
     // A query tile starting at q0 needs the causal mask iff q0 is before the
     // causal block of the tile's last key (no per-tile division).
     const int64_t k_last_blk = cbs > 0 ? ((k0 + kTile - 1) / cbs) * (int64_t)cbs : 0;
+    const float sc = p.scale_log2;
     int n = 0;
     bool ok = true;
     if (!dead) {
@@ -341,93 +345,91 @@ __global__ void __launch_bounds__(384, 1)
         if (!(ok = ra_wait_warp(bar(L::B_QF + st), (n / L::NS) & 1, abort_flag))) break;
         if (!(ok = ra_wait_warp(bar(L::B_SFULL + s), (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(slot + L::SLOT_ST, sr);
-        tmem_ld32(slot + L::SLOT_ST + 32, sr + 32);
+        uint32_t sr[32];
+        tmem_ld32(slot + L::SLOT_ST + c0, sr);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 64; ++c) reg_fence(sr[c]);
+        for (int c = 0; c < 32; ++c) reg_fence(sr[c]);
         float* x = reinterpret_cast<float*>(sr);
-        const float* lse2 = reinterpret_cast<const float*>(gbase + L::OFF_LD + st * L::LD_BYTES);
-        const float* dlt = lse2 + L::QT;
+        const float* nl = reinterpret_cast<const float*>(gbase + L::OFF_LD + st * L::LD_BYTES) + c0;   // -lse*log2e
+        const float* nd = nl + L::QT;                                                                 // -Delta
+        // x = S * log2(e)/sqrt(D) + bias(key) - lse(query) * log2(e), two columns per instruction
 #pragma unroll
-        for (int c = 0; c < 64; ++c) x[c] = fmaf(x[c], p.scale_log2, brow - lse2[c]);
+        for (int c = 0; c < 32; c += 2) {
+          float b0 = nl[c], b1 = nl[c + 1];
+          if (use_bias) fadd2(b0, b1, b0, b1, brow, brow);
+          ffma2(x[c], x[c + 1], x[c], x[c + 1], sc, sc, b0, b1);
+        }
         // per-element mask on causal-diagonal / ragged / mixed-segment tiles
         const int4 qm = meta_b ? load_meta(meta_b + q0 / kTile) : make_int4(0, 0, 3, 0);
         const bool need_causal = cbs > 0 && q0 < k_last_blk;
         const bool need_ragged = (q0 + L::QT > S) || (k0 + kTile > S);
         const bool need_seg = use_seg && !(qm.x == qm.y && km.x == km.y && qm.x == km.x);
         if (need_causal || need_ragged || need_seg || !row_valid) {
-          const int64_t cmin64 = i_first - q0;                   // visible iff c >= cmin
-          const int cmin = cmin64 < 0 ? 0 : (cmin64 > 64 ? 64 : (int)cmin64);
-          const int64_t cmax64 = S - q0;                         // valid iff c < cmax
-          const int cmax = row_valid ? (cmax64 > 64 ? 64 : (int)cmax64) : 0;
-          uint32_t vb0 = ~0u, vb1 = ~0u;
+          const int64_t cmin64 = i_first - (q0 + c0);              // visible iff c >= cmin
+          const int cmin = cmin64 < 0 ? 0 : (cmin64 > 32 ? 32 : (int)cmin64);
+          const int64_t cmax64 = S - (q0 + c0);                    // valid iff c < cmax
+          const int cmax = row_valid ? (cmax64 > 32 ? 32 : (cmax64 < 0 ? 0 : (int)cmax64)) : 0;
+          uint32_t vb = ~0u;
           if (need_seg) {
             const int32_t* sp = p.seg + b * p.seg_sb;
-            vb0 = 0;
-            vb1 = 0;
+            vb = 0;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const int64_t i = q0 + c < S ? q0 + c : S - 1;
-              vb0 |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << c;
-            }
-            asm volatile("" ::: "memory");
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              const int64_t i = q0 + 32 + c < S ? q0 + 32 + c : S - 1;
-              vb1 |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << c;
+              const int64_t i = q0 + c0 + c < S ? q0 + c0 + c : S - 1;
+              vb |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << c;
             }
           }
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const uint32_t bit = c < 32 ? (vb0 >> c) & 1u : (vb1 >> (c - 32)) & 1u;
-            const bool vis = c >= cmin && c < cmax && bit;
+          for (int c = 0; c < 32; ++c) {
+            const bool vis = c >= cmin && c < cmax && ((vb >> c) & 1u);
             x[c] = vis ? x[c] : -INFINITY;
           }
         }
-        float pr[64];
+        float pr[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) pr[c] = ex2_approx(x[c]);
+        for (int c = 0; c < 32; ++c) pr[c] = ex2_approx(x[c]);
         if (!(ok = ra_wait_warp(bar(L::B_DPFULL + s), (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
-        uint32_t dr[64];
-        tmem_ld32(slot + L::SLOT_DPT, dr);
-        tmem_ld32(slot + L::SLOT_DPT + 32, dr + 32);
+        uint32_t dr[32];
+        tmem_ld32(slot + L::SLOT_DPT + c0, dr);
         tmem_ld_wait();
 #pragma unroll
-        for (int c = 0; c < 64; ++c) reg_fence(dr[c]);
-        uint32_t pp[32], dd[32];
+        for (int c = 0; c < 32; ++c) reg_fence(dr[c]);
+        uint32_t pp[16], dd[16];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float ds0 = pr[c] * (__uint_as_float(dr[c]) - dlt[c]);
-          const float ds1 = pr[c + 1] * (__uint_as_float(dr[c + 1]) - dlt[c + 1]);
+        for (int c = 0; c < 32; c += 2) {
+          float t0, t1, ds0, ds1;
+          fadd2(t0, t1, __uint_as_float(dr[c]), __uint_as_float(dr[c + 1]), nd[c], nd[c + 1]);   // dP - Delta
+          fmul2(ds0, ds1, pr[c], pr[c + 1], t0, t1);
           pp[c >> 1] = pack_bf16x2(pr[c], pr[c + 1]);
           dd[c >> 1] = pack_bf16x2(ds0, ds1);
         }
-        // P^T and dS^T into this slot (its S^T / first half was read above).
-        tmem_st32(slot + L::SLOT_PT, pp);
-        tmem_st32(slot + L::SLOT_DST, dd);
+        // P^T and dS^T (bf16, two per column) into this slot's first half.
+        tmem_st16(slot + L::SLOT_PT + c0 / 2, pp);
+        tmem_st16(slot + L::SLOT_DST + c0 / 2, dd);
         // dS^T into shared memory for dQ^T = K^T dS^T (MN-major, 128-byte swizzle):
         // key row `row` is one 128-byte line; 16-byte chunk c lands at c ^ (row % 8).
         const uint32_t line = sbase + L::OFF_DS + s * L::DS_BYTES + row * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(line + ((c ^ (row & 7)) << 4), dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = half * 4 + c;
+          st_shared_v4(line + ((chunk ^ (row & 7)) << 4), dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+        }
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(bar(L::B_DSREADY + s));
       }
     }
-    // ---------------------------------------------------------- dK / dV epilogue
+    // ---------------------------------------------------------- epilogue: dK (columns group 0) or dV (group 1)
     bool have = n > 0 && ok;
     if (have) have = ra_wait(bar(L::B_FINAL), 0, abort_flag);
     have = __all_sync(0xffffffffu, have);
     n = __shfl_sync(0xffffffffu, n, 0);
     tc_fence_after();
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {
+    {
+      const int which = half;
       const uint32_t col = which == 0 ? L::COL_DK : L::COL_DV;
       const float mul = which == 0 ? p.scale : 1.f;
       char* base = static_cast<char*>(which == 0 ? p.dk : p.dv);
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------ dQ readout: thread = head-dim lane d
     const int sub = warp & 3;
     const int d = sub * 32 + lane;
@@ -492,6 +494,14 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 64; ++c) reg_fence(r[c]);
         tc_fence_before();
         mbar_arrive(bar(L::B_SLOTFREE + s));
+        // The previous tile's bulk reduce must have read the staging tile before
+        // it is rewritten; that wait comes only now, after the TMEM slot was
+        // released, so the next S^T / dP^T never waits on the reduction.
+        if (leader && pending) {
+          bulk_wait_group_read0();
+          mbar_arrive(bar(L::B_DQSFREE));
+          pending = false;
+        }
         // staging tile [query c][d]: a warp writes 32 consecutive floats per row
         if (n > 0 && !ra_wait_warp(bar(L::B_DQSFREE), (n - 1) & 1, abort_flag)) break;
 #pragma unroll
@@ -504,8 +514,6 @@ __global__ void __launch_bounds__(384, 1)
           tma_reduce_add_3d(&tm_dq, dqs, 0, q * L::QT, bh);
           bulk_commit_group();
           pending = true;
-          bulk_wait_group_read0();
-          mbar_arrive(bar(L::B_DQSFREE));
         }
       }
     }

@@ -13,6 +13,7 @@
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include "ptx.cuh"
 #include "ra_common.cuh"
 
 namespace ra {
@@ -399,6 +400,25 @@ __global__ void lse_merge_kernel(const MergeArgs a) {
   a.lo[b * a.lo_sb + h * a.lo_sh + i * a.lo_ss] = lse;
 }
 
+// ---------------------------------------------------------------- failure-path self-test
+
+// One warp waits, through the same bounded wait the attention kernels use, on
+// an mbarrier phase that nothing ever completes.  The wait must give up after
+// `budget` cycles, record RA_ERR_DEVICE_TIMEOUT in the status word, raise the
+// block's abort flag (checked by the remaining lanes) and return.
+__global__ void selftest_timeout_kernel(long long budget, int* gave_up) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = ra_wait_budget(smem_u32(&bar), 0, &abort_flag, budget);
+  if (threadIdx.x == 0) *gave_up = ok ? 0 : 1;
+}
+
 // ---------------------------------------------------------------- backward
 
 struct BwdPreArgs {
@@ -414,10 +434,11 @@ struct BwdPreArgs {
 };
 
 // Backward preprocess, one warp per (b, h, i) row of the padded [B*H][s_pad]
-// layout: Delta_i = <dO_i, O_i> (fp32), lse2_i = lse_i * log2(e) (+inf for a
-// row with no visible key, so its probabilities come out as 0), and the row
-// of the fp32 dQ accumulator set to zero.  Padding rows get Delta = 0 and
-// lse2 = +inf.
+// layout, written negated for the backward kernels' fused multiply-adds:
+// delta = -<dO_i, O_i> (fp32) and lse2 = -lse_i * log2(e) (-inf for a row
+// with no visible key, so its probabilities come out as 0); the row of the
+// fp32 dQ accumulator is set to zero.  Padding rows get delta = 0 and
+// lse2 = -inf.
 __global__ void bwd_pre_kernel(const BwdPreArgs a) {
   const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -429,7 +450,7 @@ __global__ void bwd_pre_kernel(const BwdPreArgs a) {
   if (i >= a.S) {
     if (lane == 0) {
       a.delta[row] = 0.f;
-      a.lse2[row] = CUDART_INF_F;
+      a.lse2[row] = -CUDART_INF_F;
     }
     return;
   }
@@ -447,9 +468,9 @@ __global__ void bwd_pre_kernel(const BwdPreArgs a) {
   }
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) {
-    a.delta[row] = s;
+    a.delta[row] = -s;
     const float l = a.lse[b * a.lse_sb + h * a.lse_sh + i * a.lse_ss];
-    a.lse2[row] = l == -CUDART_INF_F ? CUDART_INF_F : l * 1.4426950408889634f;
+    a.lse2[row] = l == -CUDART_INF_F ? -CUDART_INF_F : -l * 1.4426950408889634f;
   }
 }
 
@@ -482,7 +503,7 @@ struct SimtBwdArgs {
   MaskArgs mk;
   View4 q, k, v, dO;
   const float* lse; int64_t lse_sb, lse_sh, lse_ss;
-  const float* delta;    // [B*H][s_pad]
+  const float* delta;    // [B*H][s_pad], negated: -<dO_i, O_i>
   int64_t s_pad;
   OutView4 dq, dk, dv;
   int out_bf16;          // gradient element type: 1 bf16, 0 fp32
@@ -519,7 +540,7 @@ __global__ void __launch_bounds__(64) simt_bwd_dq_kernel(const SimtBwdArgs a) {
   const T* q = static_cast<const T*>(a.q.p) + b * a.q.sb + i * a.q.ss + h * a.q.sh;
   const T* dO = static_cast<const T*>(a.dO.p) + b * a.dO.sb + i * a.dO.ss + h * a.dO.sh;
   const float lse = a.lse[b * a.lse_sb + h * a.lse_sh + i * a.lse_ss];
-  const float dl = a.delta[(int64_t)blockIdx.y * a.s_pad + i];
+  const float dl = -a.delta[(int64_t)blockIdx.y * a.s_pad + i];
   float acc[D];
 #pragma unroll
   for (int e = 0; e < D; ++e) acc[e] = 0.f;
@@ -571,7 +592,7 @@ __global__ void __launch_bounds__(64) simt_bwd_dkdv_kernel(const SimtBwdArgs a) 
       dp = fmaf(to_f<T>(dO[e]), to_f<T>(v[e]), dp);
     }
     const float p = expf(s * a.scale + bj - lse);
-    const float ds = p * (dp - a.delta[(int64_t)blockIdx.y * a.s_pad + i]) * a.scale;
+    const float ds = p * (dp + a.delta[(int64_t)blockIdx.y * a.s_pad + i]) * a.scale;
 #pragma unroll
     for (int e = 0; e < D; ++e) {
       dv[e] = fmaf(p, to_f<T>(dO[e]), dv[e]);

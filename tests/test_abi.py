@@ -190,3 +190,9 @@ def test_ring_schedule_custom_order_is_a_permutation():
         assert sorted(tiles) == sorted(base)
     with pytest.raises(ValueError):
         api.ring_schedule(S, P, 512, 767, None, [0, 1, 1, 2])
+
+
+def test_selftest_timeout_rejects_bad_budgets_on_host():
+    lib = _lib.load()
+    assert lib.ra_selftest_timeout(10, None) == 6          # below the allowed range
+    assert lib.ra_selftest_timeout(10 ** 10, None) == 6    # above it
