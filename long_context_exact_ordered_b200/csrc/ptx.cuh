@@ -62,6 +62,20 @@ __device__ __forceinline__ bool mbar_probe(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Waits for the phase for at most about `ns` nanoseconds, suspended in
+// hardware (no issue slots used), then reports whether it completed.
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Device-wide status word (first error wins); read back by ra_get_device_status().
 __device__ int g_ra_status;
 

@@ -30,9 +30,9 @@
 // later, after the readout group has taken dQ^T out of it.
 //
 // Overlap: with two slots the "head" products of tile n+1 (S^T, dP^T) are
-// computed while the softmax group works on tile n, and the issuing thread
-// polls both "tail ready" (dV, dK, dQ^T of the oldest tile) and "head ready"
-// (slot and query stage free) so the tensor core is fed whichever is ready.
+// computed while the softmax groups work on tile n, and the issuing thread
+// feeds the tensor core whichever is ready first: the oldest tile's tail
+// (dV, dK, dQ^T) or the next head (slot and query stage free).
 #pragma once
 
 #include <cuda.h>
@@ -265,30 +265,33 @@ __global__ void __launch_bounds__(512, 1)
         q_iter_init(it, p.rd, k0, meta_b, use_seg);
         while (q_iter_next(it, p.rd) >= 0) ++N;
       }
+      // Event loop: issue whichever is ready first, the oldest tile's tail
+      // (dV, dK, dQ^T once its P^T / dS^T are written) or the next head
+      // (S^T, dP^T once its slot and query stage are free).  Polls suspend in
+      // hardware for a few tens of nanoseconds, so this warp does not take
+      // issue slots from the softmax / readout warps of its sub-partition.
       bool ok = ra_wait(bar(L::B_KV), 0, abort_flag);
       int hd = 0, tl = 0;    // next head (S^T, dP^T) and next tail (dV, dK, dQ^T) to issue
       long long idle_since = clock64();
       while (ok && tl < N) {
         bool progress = false;
-        if (tl < hd) {
+        if (tl < hd && mbar_try_wait_ns(bar(L::B_DSREADY + (tl & 1)), (tl >> 1) & 1, 40)) {
           const int s = tl & 1;
-          if (mbar_probe(bar(L::B_DSREADY + s), (tl >> 1) & 1)) {
-            tc_fence_after();
-            const uint32_t slot = tmem + s * L::SLOT_COLS;
-            const int st = tl % L::NS;
-            issue_kv(tmem + L::COL_DV, slot + L::SLOT_PT, sbase + L::OFF_DO + st * L::Q_BYTES, tl > 0);
-            issue_kv(tmem + L::COL_DK, slot + L::SLOT_DST, sbase + L::OFF_Q + st * L::Q_BYTES, tl > 0);
-            issue_dq(slot + L::SLOT_DQT, sbase + L::OFF_DS + s * L::DS_BYTES);
-            mma_commit(bar(L::B_DQFULL + s));
-            mma_commit(bar(L::B_QE + st));
-            ++tl;
-            progress = true;
-          }
+          tc_fence_after();
+          const uint32_t slot = tmem + s * L::SLOT_COLS;
+          const int st = tl % L::NS;
+          issue_kv(tmem + L::COL_DV, slot + L::SLOT_PT, sbase + L::OFF_DO + st * L::Q_BYTES, tl > 0);
+          issue_kv(tmem + L::COL_DK, slot + L::SLOT_DST, sbase + L::OFF_Q + st * L::Q_BYTES, tl > 0);
+          issue_dq(slot + L::SLOT_DQT, sbase + L::OFF_DS + s * L::DS_BYTES);
+          mma_commit(bar(L::B_DQFULL + s));
+          mma_commit(bar(L::B_QE + st));
+          ++tl;
+          progress = true;
         }
         if (hd < N && hd < tl + L::NSLOT) {
           const int s = hd & 1, st = hd % L::NS;
-          const bool slot_free = hd < L::NSLOT || mbar_probe(bar(L::B_SLOTFREE + s), ((hd >> 1) - 1) & 1);
-          if (slot_free && mbar_probe(bar(L::B_QF + st), (hd / L::NS) & 1)) {
+          const bool slot_free = hd < L::NSLOT || mbar_try_wait_ns(bar(L::B_SLOTFREE + s), ((hd >> 1) - 1) & 1, 40);
+          if (slot_free && mbar_try_wait_ns(bar(L::B_QF + st), (hd / L::NS) & 1, 40)) {
             tc_fence_after();
             const uint32_t slot = tmem + s * L::SLOT_COLS;
             issue_sd(slot + L::SLOT_ST, ka, sbase + L::OFF_Q + st * L::Q_BYTES);
