@@ -361,9 +361,11 @@ def blas_threads():
 
 def cpu_baseline(w, budget_s=20.0):
     """The oracle as it stands on this host's cores, on a bounded sample of the workload."""
-    secs, pairs = oracle_sample(w, 8, [0], seed=1)                 # calibration
-    per_row = secs / 8
-    rows = int(max(8, min(4096, budget_s / max(per_row, 1e-6))))
+    # two-point calibration: the head's float64 conversion is a fixed cost per sample
+    t8, _ = oracle_sample(w, 8, [0], seed=1)
+    t64, _ = oracle_sample(w, 64, [0], seed=1)
+    per_row = max((t64 - t8) / 56, 1e-6)
+    rows = int(max(8, min(8192, (budget_s - t8) / per_row)))
     secs, pairs = oracle_sample(w, rows, [0], seed=2)
     val = 14.0 * w.D * pairs / secs / 1e12
     return {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",

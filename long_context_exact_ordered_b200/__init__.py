@@ -17,12 +17,13 @@ from .api import (  # noqa: F401
     ringattention_backward,
     ringattention_static,
     selftest_timeout,
+    visible_count_probe,
     workspace_size,
 )
 from ._lib import RingAttnError, load  # noqa: F401
 
 __all__ = [
     "ringattention", "ringattention_backward", "ringattention_static", "ring_step", "init_state", "finalize", "lse_merge",
-    "device_status", "selftest_timeout", "count_visible_pairs", "ring_schedule", "workspace_size", "RingAttentionFunction",
+    "device_status", "selftest_timeout", "count_visible_pairs", "ring_schedule", "workspace_size", "RingAttentionFunction", "visible_count_probe",
     "RingAttnError", "load",
 ]

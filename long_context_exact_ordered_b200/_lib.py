@@ -10,6 +10,8 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libringattn.so")
+# Debug build (-DRA_DEBUG_COUNT): same entry points plus ra_debug_set_counts.
+COUNT_LIB_PATH = os.path.join(HERE, "libringattn_count.so")
 
 RA_F32, RA_BF16, RA_I32 = 0, 1, 2
 RA_MAX_RING = 64
@@ -85,6 +87,34 @@ def load() -> ctypes.CDLL:
             fn.argtypes = args
         _lib = lib
     return _lib
+
+
+_count_lib = None
+
+
+def load_count() -> ctypes.CDLL:
+    """Load the debug build (kernels that also count visible pairs); raise if absent."""
+    global _count_lib
+    if _count_lib is None:
+        if not os.path.exists(COUNT_LIB_PATH):
+            raise ImportError(f"{COUNT_LIB_PATH} is missing: build it with `python -m long_context_exact_ordered_b200.build`")
+        lib = ctypes.CDLL(COUNT_LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        lib.ra_debug_set_counts.restype = ctypes.c_int
+        lib.ra_debug_set_counts.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        _count_lib = lib
+    return _count_lib
+
+
+def swap(lib):
+    """Make ``lib`` the library every later call goes to; return the previous one."""
+    global _lib
+    prev = load()
+    _lib = lib
+    return prev
 
 
 class RingAttnError(RuntimeError):

@@ -9,10 +9,12 @@ attention_bias, segment_ids, blockwise_kwargs)``).
 
 from __future__ import annotations
 
+import contextlib
 import ctypes
 
 import torch
 
+from . import _lib
 from ._lib import RA_BF16, RA_F32, RA_I32, RA_MAX_RING, RaParams, RaTensor, check, load
 
 _DT = {torch.float32: RA_F32, torch.bfloat16: RA_BF16, torch.int32: RA_I32}
@@ -276,3 +278,26 @@ class RingAttentionFunction(torch.autograd.Function):
         q, k, v, o, lse, bias, seg = ctx.saved_tensors
         dq, dk, dv = ringattention_backward(q, k, v, o, lse, do.contiguous(), bias, seg, **ctx.kwargs)
         return dq, dk, dv, None, None, None
+
+
+@contextlib.contextmanager
+def visible_count_probe(fwd_row_counts=None, bwd_col_counts=None):
+    """Inside the block, calls run the debug build of the library, whose
+    tensor-core kernels record how many pairs their own skipping and masking
+    let into the softmax: per query row in ``fwd_row_counts`` (int32
+    [B, H, S], overwritten by each forward) and per key in ``bwd_col_counts``
+    (int32 [B, H, S], added to by each backward: zero it first).  For the
+    mask bit-exactness tests only."""
+    for t in (fwd_row_counts, bwd_col_counts):
+        if t is not None and (t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("count buffers must be contiguous int32 CUDA tensors")
+    dbg = _lib.load_count()
+    check(dbg.ra_debug_set_counts(None if fwd_row_counts is None else fwd_row_counts.data_ptr(),
+                                  None if bwd_col_counts is None else bwd_col_counts.data_ptr()),
+          "ra_debug_set_counts")
+    prev = _lib.swap(dbg)
+    try:
+        yield
+    finally:
+        _lib.swap(prev)
+        dbg.ra_debug_set_counts(None, None)

@@ -27,6 +27,13 @@ static __device__ __align__(256) unsigned char g_ra_static_scratch[RA_STATIC_SCR
 // Written only by the failure-path self-test kernel (1 = its wait gave up).
 static __device__ int g_ra_selftest_result;
 
+#ifdef RA_DEBUG_COUNT
+#include "../../include/ringattn_debug.h"
+// Count buffers of the debug build (set by ra_debug_set_counts; null = off).
+static int32_t* g_dbg_fwd_rows = nullptr;
+static int32_t* g_dbg_bwd_cols = nullptr;
+#endif
+
 namespace {
 
 // ---------------------------------------------------------------- validation
@@ -268,6 +275,9 @@ int launch_fwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v,
   prm.bias_sb = mk.bias_sb;
   prm.bias_ss = mk.bias_ss;
   prm.meta = meta;
+#ifdef RA_DEBUG_COUNT
+  prm.dbg_count = g_dbg_fwd_rows;
+#endif
   const int64_t grid = (int64_t)prm.npairs * prm.B * prm.H;
   if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(ra_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
@@ -351,6 +361,9 @@ int launch_bwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v,
   prm.bias_sb = mk.bias_sb;
   prm.bias_ss = mk.bias_ss;
   prm.meta = meta;
+#ifdef RA_DEBUG_COUNT
+  prm.dbg_count = g_dbg_bwd_cols;
+#endif
   const int64_t grid = (int64_t)rd.ntiles * prm.B * prm.H;
   if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
   if (cudaFuncSetAttribute(ra_bwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
@@ -741,6 +754,14 @@ int ra_selftest_timeout(int64_t budget_cycles, void* stream) {
   selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_cycles, ptr);
   return last_cuda();
 }
+
+#ifdef RA_DEBUG_COUNT
+int ra_debug_set_counts(int32_t* fwd_row_counts, int32_t* bwd_col_counts) {
+  g_dbg_fwd_rows = fwd_row_counts;
+  g_dbg_bwd_cols = bwd_col_counts;
+  return RA_OK;
+}
+#endif
 
 int ra_get_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RA_ERR_CUDA;

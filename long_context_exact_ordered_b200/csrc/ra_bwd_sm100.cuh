@@ -69,11 +69,11 @@ struct BwdLayout {
   static constexpr int B_QE = B_QF + NS;          // [NS] query stage free
   static constexpr int B_SFULL = B_QE + NS;       // [NSLOT] S^T computed
   static constexpr int B_DPFULL = B_SFULL + NSLOT;   // [NSLOT] dP^T computed
-  static constexpr int B_DSREADY = B_DPFULL + NSLOT; // [NSLOT] P^T, dS^T written (256 arrivals)
+  static constexpr int B_DSREADY = B_DPFULL + NSLOT; // [NSLOT] P^T, dS^T written (8 arrivals: softmax warps)
   static constexpr int B_DQFULL = B_DSREADY + NSLOT; // [NSLOT] dQ^T computed
-  static constexpr int B_SLOTFREE = B_DQFULL + NSLOT;  // [NSLOT] dQ^T read out (128 arrivals)
+  static constexpr int B_SLOTFREE = B_DQFULL + NSLOT;  // [NSLOT] dQ^T read out (4 arrivals: readout warps)
   static constexpr int B_FINAL = B_SLOTFREE + NSLOT;
-  static constexpr int B_DQSFULL = B_FINAL + 1;      // staging written (128 arrivals)
+  static constexpr int B_DQSFULL = B_FINAL + 1;      // staging written (4 arrivals)
   static constexpr int B_DQSFREE = B_DQSFULL + 1;    // staging read by the bulk reduce
   static constexpr int NBAR = B_DQSFREE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -107,6 +107,7 @@ struct BwdParams {
   const float* bias;
   int64_t bias_sb, bias_ss;
   const int4* meta;
+  int32_t* dbg_count;        // RA_DEBUG_COUNT builds: visible queries per key, [B, H, S], pre-zeroed
 };
 
 // Tensor bulk reduce-add shared -> global (3-D tile, fp32 add), tracked by a bulk group.
@@ -168,12 +169,12 @@ __global__ void __launch_bounds__(512, 1)
     for (int i = 0; i < L::NSLOT; ++i) {
       mbar_init(bar(L::B_SFULL + i), 1);
       mbar_init(bar(L::B_DPFULL + i), 1);
-      mbar_init(bar(L::B_DSREADY + i), 256);
+      mbar_init(bar(L::B_DSREADY + i), 8);     // one arrive per softmax warp
       mbar_init(bar(L::B_DQFULL + i), 1);
-      mbar_init(bar(L::B_SLOTFREE + i), 128);
+      mbar_init(bar(L::B_SLOTFREE + i), 4);    // one arrive per readout warp
     }
     mbar_init(bar(L::B_FINAL), 1);
-    mbar_init(bar(L::B_DQSFULL), 128);
+    mbar_init(bar(L::B_DQSFULL), 4);
     mbar_init(bar(L::B_DQSFREE), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -231,32 +232,37 @@ __global__ void __launch_bounds__(512, 1)
         if (i >= 0) ra_wait_drain(bar(L::B_QF + i % L::NS), (i / L::NS) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (event loop)
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, L::QT, false, false);
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, L::QT, true, true);
       const uint32_t ka = sbase + L::OFF_K, va = sbase + L::OFF_V;
-      auto issue_sd = [&](uint32_t d_tmem, uint32_t a_base, uint32_t b_base) {   // S^T or dP^T
+      // Descriptors are built once per operand tile; the K-step offsets are
+      // added to the start-address field (address >> 4, no carry: shared
+      // memory ends below 2^18 bytes), keeping the issue loop short.
+      const uint64_t ka_k = smem_desc_sw128(ka, 16, 1024), va_k = smem_desc_sw128(va, 16, 1024);
+      const uint64_t ka_mn = smem_desc_sw128(ka, L::KV_CHUNK, 1024);
+      auto issue_sd = [&](uint32_t d_tmem, uint64_t a_desc, uint32_t b_base) {   // S^T or dP^T
+        const uint64_t b_desc = smem_desc_sw128(b_base, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t oa = (kk / 4) * L::KV_CHUNK + (kk % 4) * 32;
-          const uint32_t ob = (kk / 4) * L::Q_CHUNK + (kk % 4) * 32;
-          mma_ss(d_tmem, smem_desc_sw128(a_base + oa, 16, 1024), smem_desc_sw128(b_base + ob, 16, 1024), IDESC_SD,
-                 kk > 0);
+          const uint32_t oa = ((kk / 4) * L::KV_CHUNK + (kk % 4) * 32) >> 4;
+          const uint32_t ob = ((kk / 4) * L::Q_CHUNK + (kk % 4) * 32) >> 4;
+          mma_ss(d_tmem, a_desc + oa, b_desc + ob, IDESC_SD, kk > 0);
         }
       };
       auto issue_kv = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool acc) {   // dV or dK
+        const uint64_t b_desc = smem_desc_sw128(b_base, L::Q_CHUNK, 1024);
 #pragma unroll
         for (int kk = 0; kk < L::QT / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, smem_desc_sw128(b_base + kk * 2048, L::Q_CHUNK, 1024), IDESC_KV,
-                 (acc || kk > 0) ? 1u : 0u);
+          mma_ts(d_tmem, a_tmem + kk * 8, b_desc + kk * (2048 >> 4), IDESC_KV, (acc || kk > 0) ? 1u : 0u);
       };
       auto issue_dq = [&](uint32_t d_tmem, uint32_t ds_base) {
+        const uint64_t b_desc = smem_desc_sw128(ds_base, L::DS_BYTES, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ss(d_tmem, smem_desc_sw128(ka + kk * 2048, L::KV_CHUNK, 1024),
-                 smem_desc_sw128(ds_base + kk * 2048, L::DS_BYTES, 1024), IDESC_DQ, kk > 0);
+          mma_ss(d_tmem, ka_mn + kk * (2048 >> 4), b_desc + kk * (2048 >> 4), IDESC_DQ, kk > 0);
       };
       // number of query tiles this key tile visits
       int N = 0;
@@ -265,52 +271,43 @@ __global__ void __launch_bounds__(512, 1)
         q_iter_init(it, p.rd, k0, meta_b, use_seg);
         while (q_iter_next(it, p.rd) >= 0) ++N;
       }
-      // Event loop: issue whichever is ready first, the oldest tile's tail
-      // (dV, dK, dQ^T once its P^T / dS^T are written) or the next head
-      // (S^T, dP^T once its slot and query stage are free).  Polls suspend in
-      // hardware for a few tens of nanoseconds, so this warp does not take
-      // issue slots from the softmax / readout warps of its sub-partition.
+      // Issue order (two TMEM slots, tile n in slot n % 2):
+      //   S^T(0) dP^T(0) S^T(1) dP^T(1) | tail(0) S^T(2) dP^T(2) | tail(1) S^T(3) dP^T(3) | ...
+      // with tail(n) = dQ^T(n), then dV(n), dK(n).  The tensor pipe runs one
+      // thread's MMAs in issue order, so S^T(n+2) may follow tail(n) at once
+      // (it overwrites P^T / dS^T(n) only after dV / dK(n) have read them);
+      // dP^T(n+2) overwrites dQ^T(n) and waits for its readout, which runs
+      // while dV, dK(n) and S^T(n+2) execute.  The softmax of tile n+1 has
+      // tail(n), S^T(n+2) and dP^T(n+2) of tensor work to hide behind.
       bool ok = ra_wait(bar(L::B_KV), 0, abort_flag);
-      int hd = 0, tl = 0;    // next head (S^T, dP^T) and next tail (dV, dK, dQ^T) to issue
-      long long idle_since = clock64();
-      while (ok && tl < N) {
-        bool progress = false;
-        if (tl < hd && mbar_try_wait_ns(bar(L::B_DSREADY + (tl & 1)), (tl >> 1) & 1, 40)) {
-          const int s = tl & 1;
-          tc_fence_after();
-          const uint32_t slot = tmem + s * L::SLOT_COLS;
-          const int st = tl % L::NS;
-          issue_kv(tmem + L::COL_DV, slot + L::SLOT_PT, sbase + L::OFF_DO + st * L::Q_BYTES, tl > 0);
-          issue_kv(tmem + L::COL_DK, slot + L::SLOT_DST, sbase + L::OFF_Q + st * L::Q_BYTES, tl > 0);
-          issue_dq(slot + L::SLOT_DQT, sbase + L::OFF_DS + s * L::DS_BYTES);
-          mma_commit(bar(L::B_DQFULL + s));
-          mma_commit(bar(L::B_QE + st));
-          ++tl;
-          progress = true;
-        }
-        if (hd < N && hd < tl + L::NSLOT) {
-          const int s = hd & 1, st = hd % L::NS;
-          const bool slot_free = hd < L::NSLOT || mbar_try_wait_ns(bar(L::B_SLOTFREE + s), ((hd >> 1) - 1) & 1, 40);
-          if (slot_free && mbar_try_wait_ns(bar(L::B_QF + st), (hd / L::NS) & 1, 40)) {
-            tc_fence_after();
-            const uint32_t slot = tmem + s * L::SLOT_COLS;
-            issue_sd(slot + L::SLOT_ST, ka, sbase + L::OFF_Q + st * L::Q_BYTES);
-            mma_commit(bar(L::B_SFULL + s));
-            issue_sd(slot + L::SLOT_DPT, va, sbase + L::OFF_DO + st * L::Q_BYTES);
-            mma_commit(bar(L::B_DPFULL + s));
-            ++hd;
-            progress = true;
-          }
-        }
-        if (progress) {
-          idle_since = clock64();
-        } else if (*abort_flag) {
-          ok = false;
-        } else if (clock64() - idle_since > RA_SPIN_BUDGET) {
-          raise_status(9 /* RA_ERR_DEVICE_TIMEOUT */);
-          *abort_flag = 1;
-          ok = false;
-        }
+      auto head_s = [&](int m) -> bool {
+        const int st = m % L::NS;
+        if (!ra_wait(bar(L::B_QF + st), (m / L::NS) & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_sd(tmem + (m & 1) * L::SLOT_COLS + L::SLOT_ST, ka_k, sbase + L::OFF_Q + st * L::Q_BYTES);
+        mma_commit(bar(L::B_SFULL + (m & 1)));
+        return true;
+      };
+      auto head_dp = [&](int m) -> bool {
+        const int s = m & 1, st = m % L::NS;
+        if (m >= L::NSLOT && !ra_wait(bar(L::B_SLOTFREE + s), ((m >> 1) - 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        issue_sd(tmem + s * L::SLOT_COLS + L::SLOT_DPT, va_k, sbase + L::OFF_DO + st * L::Q_BYTES);
+        mma_commit(bar(L::B_DPFULL + s));
+        return true;
+      };
+      for (int m = 0; ok && m < N && m < L::NSLOT; ++m) ok = head_s(m) && head_dp(m);
+      for (int t = 0; ok && t < N; ++t) {
+        const int s = t & 1, st = t % L::NS;
+        if (!(ok = ra_wait(bar(L::B_DSREADY + s), (t >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t slot = tmem + s * L::SLOT_COLS;
+        issue_dq(slot + L::SLOT_DQT, sbase + L::OFF_DS + s * L::DS_BYTES);
+        mma_commit(bar(L::B_DQFULL + s));
+        issue_kv(tmem + L::COL_DV, slot + L::SLOT_PT, sbase + L::OFF_DO + st * L::Q_BYTES, t > 0);
+        issue_kv(tmem + L::COL_DK, slot + L::SLOT_DST, sbase + L::OFF_Q + st * L::Q_BYTES, t > 0);
+        mma_commit(bar(L::B_QE + st));
+        if (t + L::NSLOT < N) ok = head_s(t + L::NSLOT) && head_dp(t + L::NSLOT);
       }
       mma_commit(bar(L::B_FINAL));
       ra_wait_drain(bar(L::B_FINAL), 0);
@@ -336,6 +333,9 @@ __global__ void __launch_bounds__(512, 1)
     // causal block of the tile's last key (no per-tile division).
     const int64_t k_last_blk = cbs > 0 ? ((k0 + kTile - 1) / cbs) * (int64_t)cbs : 0;
     const float sc = p.scale_log2;
+#ifdef RA_DEBUG_COUNT
+    int dbg_vis = 0;
+#endif
     int n = 0;
     bool ok = true;
     if (!dead) {
@@ -389,6 +389,11 @@ __global__ void __launch_bounds__(512, 1)
             x[c] = vis ? x[c] : -INFINITY;
           }
         }
+#ifdef RA_DEBUG_COUNT
+        // visible pairs as decided by this kernel's own tile skipping and masking
+#pragma unroll
+        for (int c = 0; c < 32; ++c) dbg_vis += x[c] != -INFINITY;
+#endif
         float pr[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) pr[c] = ex2_approx(x[c]);
@@ -422,9 +427,16 @@ __global__ void __launch_bounds__(512, 1)
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::B_DSREADY + s));
+        // one arrive per warp: per-lane arrives on one barrier serialise in the
+        // shared-memory pipe, which the tensor cores' operand reads also use
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_DSREADY + s));
       }
     }
+#ifdef RA_DEBUG_COUNT
+    // the two column halves of a key row add their counts
+    if (row_valid && ok && p.dbg_count) atomicAdd(p.dbg_count + ((int64_t)b * p.H + h) * S + j, dbg_vis);
+#endif
     // ---------------------------------------------------------- epilogue: dK (columns group 0) or dV (group 1)
     bool have = n > 0 && ok;
     if (have) have = ra_wait(bar(L::B_FINAL), 0, abort_flag);
@@ -496,7 +508,8 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) reg_fence(r[c]);
         tc_fence_before();
-        mbar_arrive(bar(L::B_SLOTFREE + s));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_SLOTFREE + s));
         // The previous tile's bulk reduce must have read the staging tile before
         // it is rewritten; that wait comes only now, after the TMEM slot was
         // released, so the next S^T / dP^T never waits on the reduction.
@@ -510,7 +523,8 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int c = 0; c < 64; ++c) st_shared_f32(dqs + c * (D * 4) + d * 4, __uint_as_float(r[c]) * p.scale);
         fence_proxy_async_smem();
-        mbar_arrive(bar(L::B_DQSFULL));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_DQSFULL));
         if (leader) {
           if (!ra_wait(bar(L::B_DQSFULL), n & 1, abort_flag)) break;
           // rows past S fall outside the tensor map and are not written

@@ -91,6 +91,7 @@ struct FwdParams {
   const float* bias;       // [B, S] or null
   int64_t bias_sb, bias_ss;
   const int4* meta;        // [B, ntiles] or null
+  int32_t* dbg_count;      // RA_DEBUG_COUNT builds: visible keys per query row, [B, H, S]
 };
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -287,6 +288,9 @@ __global__ void __launch_bounds__(384, 1)
     KvIter it;
     kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
     float m_ref = -INFINITY, l = 0.f;
+#ifdef RA_DEBUG_COUNT
+    int dbg_vis = 0;
+#endif
     int n = 0;
     bool ok = true;
     for (int32_t t = kv_iter_next(it, p.rd); t >= 0; t = kv_iter_next(it, p.rd), ++n) {
@@ -349,6 +353,12 @@ __global__ void __launch_bounds__(384, 1)
           x[c] = vis ? x[c] : -INFINITY;
         }
       }
+#ifdef RA_DEBUG_COUNT
+      // visible pairs as decided by this kernel's own tile skipping and
+      // masking: every score still finite here enters the softmax
+#pragma unroll
+      for (int c = 0; c < 128; ++c) dbg_vis += x[c] != -INFINITY;
+#endif
       // tile max (three-input max, two independent chains)
       float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
 #pragma unroll
@@ -439,6 +449,9 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (qrow < S && ok)
       p.lse[b * p.lse_sb + h * p.lse_sh + qrow * p.lse_ss] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+#ifdef RA_DEBUG_COUNT
+    if (qrow < S && ok && p.dbg_count) p.dbg_count[((int64_t)b * p.H + h) * S + qrow] = dbg_vis;
+#endif
   }
 
   // ------------------------------------------------------------ teardown

@@ -257,6 +257,20 @@ def visible_count_rows(rows, S, causal_block_size=None, seg_b=None, bias_b=None)
     return out
 
 
+def visible_count_cols(S, causal_block_size=None, seg_b=None, bias_b=None):
+    """Exact integer number of visible query rows for each key j of one batch.
+
+    The column sums of the same mask as ``visible_count_rows`` (which keys
+    take part follows "RingAttention核心功能全解析", 核心API调用: causal_block_size,
+    segment_ids, attention_bias).
+    """
+    out = np.zeros(S, dtype=np.int64)
+    rows = np.arange(S, dtype=np.int64)
+    for a, e in _row_chunks(S, S):
+        out += visible_mask(rows[a:e], S, causal_block_size, seg_b, bias_b).sum(axis=0)
+    return out
+
+
 def visible_pairs_total(B, H, S, causal_block_size=None, segment_ids=None, attention_bias=None):
     """Exact integer count of visible (i, j) pairs summed over all (b, h).
 

@@ -16,10 +16,11 @@ import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ringattn.h")
+DEBUG_HEADER = os.path.join(ROOT, "include", "ringattn_debug.h")
 
 
-def declared_functions():
-    text = open(HEADER).read()
+def declared_functions(header=HEADER):
+    text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(ra_[a-z_]+)\s*\(", text)))
 
@@ -32,6 +33,18 @@ def test_every_declared_symbol_is_exported():
     for n in names:
         assert hasattr(lib, n), n
         assert n in _lib.SIGNATURES, n
+
+
+def test_debug_build_exports_its_extra_symbol():
+    """The RA_DEBUG_COUNT build exports everything both headers declare; the
+    release build does not carry the debug entry point."""
+    dbg = _lib.load_count()
+    extra = declared_functions(DEBUG_HEADER)
+    assert extra == ["ra_debug_set_counts"]
+    for n in declared_functions() + extra:
+        assert hasattr(dbg, n), n
+    assert not hasattr(_lib.load(), "ra_debug_set_counts")
+    assert dbg.ra_debug_set_counts(None, None) == 0
 
 
 def test_struct_layout_matches_header():

@@ -272,6 +272,31 @@ def test_visible_counts_closed_forms():
     assert oracle.visible_pairs_total(1, 2, S, None) == 2 * S * S
 
 
+def test_visible_column_counts_closed_forms():
+    """Per key j: the number of query rows that see it (what the backward's
+    debug counter is compared with), from closed forms, not from the mask."""
+    S = 200
+    j = np.arange(S)
+    np.testing.assert_array_equal(oracle.visible_count_cols(S, None), np.full(S, S))
+    np.testing.assert_array_equal(oracle.visible_count_cols(S, 1), S - j)
+    for c in (2, 7, 64):
+        # queries i with i // c >= j // c are i >= (j // c) * c
+        np.testing.assert_array_equal(oracle.visible_count_cols(S, c), S - (j // c) * c)
+    lengths = [37, 80, 1, 82]
+    seg = np.repeat(np.arange(4), lengths)
+    end = np.repeat(np.cumsum(lengths), lengths)                  # exclusive end of j's document
+    np.testing.assert_array_equal(oracle.visible_count_cols(S, 1, seg), end - j)
+    np.testing.assert_array_equal(oracle.visible_count_cols(S, None, seg), np.repeat(lengths, lengths))
+    bias = np.zeros(S)
+    bias[[0, 5, 199]] = -np.inf
+    want = (S - j).astype(np.int64)
+    want[[0, 5, 199]] = 0                                         # a -inf bias masks the key for everyone
+    np.testing.assert_array_equal(oracle.visible_count_cols(S, 1, None, bias), want)
+    # rows and columns count the same pairs
+    for c, sg, bs in ((1, seg, None), (3, None, bias), (None, seg, bias)):
+        assert oracle.visible_count_cols(S, c, sg, bs).sum() == oracle.visible_count_rows(j, S, c, sg, bs).sum()
+
+
 # --------------------------------------------------------------------------- P8 / P9
 
 def test_backward_matches_finite_differences():
