@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {   // the whole warp runs the issuer; one elected lane issues (ptx.cuh)
       constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, L::QT, false, false);
       constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);
       constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, L::QT, true, true);
@@ -249,20 +249,20 @@ __global__ void __launch_bounds__(512, 1)
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oa = ((kk / 4) * L::KV_CHUNK + (kk % 4) * 32) >> 4;
           const uint32_t ob = ((kk / 4) * L::Q_CHUNK + (kk % 4) * 32) >> 4;
-          mma_ss(d_tmem, a_desc + oa, b_desc + ob, IDESC_SD, kk > 0);
+          mma_ss_w(d_tmem, a_desc + oa, b_desc + ob, IDESC_SD, kk > 0);
         }
       };
       auto issue_kv = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool acc) {   // dV or dK
         const uint64_t b_desc = smem_desc_sw128(b_base, L::Q_CHUNK, 1024);
 #pragma unroll
         for (int kk = 0; kk < L::QT / 16; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, b_desc + kk * (2048 >> 4), IDESC_KV, (acc || kk > 0) ? 1u : 0u);
+          mma_ts_w(d_tmem, a_tmem + kk * 8, b_desc + kk * (2048 >> 4), IDESC_KV, (acc || kk > 0) ? 1u : 0u);
       };
       auto issue_dq = [&](uint32_t d_tmem, uint32_t ds_base) {
         const uint64_t b_desc = smem_desc_sw128(ds_base, L::DS_BYTES, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ss(d_tmem, ka_mn + kk * (2048 >> 4), b_desc + kk * (2048 >> 4), IDESC_DQ, kk > 0);
+          mma_ss_w(d_tmem, ka_mn + kk * (2048 >> 4), b_desc + kk * (2048 >> 4), IDESC_DQ, kk > 0);
       };
       // number of query tiles this key tile visits
       int N = 0;
@@ -279,37 +279,37 @@ __global__ void __launch_bounds__(512, 1)
       // dP^T(n+2) overwrites dQ^T(n) and waits for its readout, which runs
       // while dV, dK(n) and S^T(n+2) execute.  The softmax of tile n+1 has
       // tail(n), S^T(n+2) and dP^T(n+2) of tensor work to hide behind.
-      bool ok = ra_wait(bar(L::B_KV), 0, abort_flag);
+      bool ok = ra_wait_warp(bar(L::B_KV), 0, abort_flag);
       auto head_s = [&](int m) -> bool {
         const int st = m % L::NS;
-        if (!ra_wait(bar(L::B_QF + st), (m / L::NS) & 1, abort_flag)) return false;
+        if (!ra_wait_warp(bar(L::B_QF + st), (m / L::NS) & 1, abort_flag)) return false;
         tc_fence_after();
         issue_sd(tmem + (m & 1) * L::SLOT_COLS + L::SLOT_ST, ka_k, sbase + L::OFF_Q + st * L::Q_BYTES);
-        mma_commit(bar(L::B_SFULL + (m & 1)));
+        mma_commit_w(bar(L::B_SFULL + (m & 1)));
         return true;
       };
       auto head_dp = [&](int m) -> bool {
         const int s = m & 1, st = m % L::NS;
-        if (m >= L::NSLOT && !ra_wait(bar(L::B_SLOTFREE + s), ((m >> 1) - 1) & 1, abort_flag)) return false;
+        if (m >= L::NSLOT && !ra_wait_warp(bar(L::B_SLOTFREE + s), ((m >> 1) - 1) & 1, abort_flag)) return false;
         tc_fence_after();
         issue_sd(tmem + s * L::SLOT_COLS + L::SLOT_DPT, va_k, sbase + L::OFF_DO + st * L::Q_BYTES);
-        mma_commit(bar(L::B_DPFULL + s));
+        mma_commit_w(bar(L::B_DPFULL + s));
         return true;
       };
       for (int m = 0; ok && m < N && m < L::NSLOT; ++m) ok = head_s(m) && head_dp(m);
       for (int t = 0; ok && t < N; ++t) {
         const int s = t & 1, st = t % L::NS;
-        if (!(ok = ra_wait(bar(L::B_DSREADY + s), (t >> 1) & 1, abort_flag))) break;
+        if (!(ok = ra_wait_warp(bar(L::B_DSREADY + s), (t >> 1) & 1, abort_flag))) break;
         tc_fence_after();
         const uint32_t slot = tmem + s * L::SLOT_COLS;
         issue_dq(slot + L::SLOT_DQT, sbase + L::OFF_DS + s * L::DS_BYTES);
-        mma_commit(bar(L::B_DQFULL + s));
+        mma_commit_w(bar(L::B_DQFULL + s));
         issue_kv(tmem + L::COL_DV, slot + L::SLOT_PT, sbase + L::OFF_DO + st * L::Q_BYTES, t > 0);
         issue_kv(tmem + L::COL_DK, slot + L::SLOT_DST, sbase + L::OFF_Q + st * L::Q_BYTES, t > 0);
-        mma_commit(bar(L::B_QE + st));
+        mma_commit_w(bar(L::B_QE + st));
         if (t + L::NSLOT < N) ok = head_s(t + L::NSLOT) && head_dp(t + L::NSLOT);
       }
-      mma_commit(bar(L::B_FINAL));
+      mma_commit_w(bar(L::B_FINAL));
       ra_wait_drain(bar(L::B_FINAL), 0);
     }
     __syncwarp();

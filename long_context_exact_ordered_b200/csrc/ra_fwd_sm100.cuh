@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    {   // the whole warp runs the issuer; one elected lane issues (ptx.cuh)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
       const uint32_t tS[2] = {tmem + L::COL_S0, tmem + L::COL_S1};
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * L::CHUNK_BYTES + (kk % 4) * 32;
-          mma_ss(tS[qt], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), IDESC_S,
+          mma_ss_w(tS[qt], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), IDESC_S,
                  kk > 0);
         }
       };
@@ -205,59 +205,59 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t va = sbase + L::OFF_V + vs * L::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk)
-          mma_ts(tO[qt], tS[qt] + kk * 8, smem_desc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), IDESC_PV,
+          mma_ts_w(tO[qt], tS[qt] + kk * 8, smem_desc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), IDESC_PV,
                  (acc || kk > 0) ? 1u : 0u);
       };
       KvIter it;
       kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
       int32_t t = kv_iter_next(it, p.rd);
-      bool ok = ra_wait(bar(L::B_Q), 0, abort_flag);
+      bool ok = ra_wait_warp(bar(L::B_Q), 0, abort_flag);
       if (ok && t >= 0) {
-        ok = ra_wait(bar(L::B_KFULL + 0), 0, abort_flag);
+        ok = ra_wait_warp(bar(L::B_KFULL + 0), 0, abort_flag);
         if (ok) {
           tc_fence_after();
           issue_s(0, 0);
-          mma_commit(bar(L::B_SFULL + 0));
+          mma_commit_w(bar(L::B_SFULL + 0));
           issue_s(1, 0);
-          mma_commit(bar(L::B_SFULL + 1));
-          mma_commit(bar(L::B_KEMPTY + 0));
+          mma_commit_w(bar(L::B_SFULL + 1));
+          mma_commit_w(bar(L::B_KEMPTY + 0));
         }
         for (int n = 0; ok; ++n) {
           const int32_t tn = kv_iter_next(it, p.rd);
           const bool last = tn < 0;
           const int vs = n % L::VS, ks1 = (n + 1) % L::KS;
           const uint32_t ph = n & 1;
-          if (!(ok = ra_wait(bar(L::B_VFULL + vs), (n / L::VS) & 1, abort_flag))) break;
+          if (!(ok = ra_wait_warp(bar(L::B_VFULL + vs), (n / L::VS) & 1, abort_flag))) break;
           // query tile 0
-          if (!(ok = ra_wait(bar(L::B_PFULL + 0), ph, abort_flag))) break;
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 0), ph, abort_flag))) break;
           tc_fence_after();
           issue_pv(0, vs, n > 0);
-          mma_commit(bar(L::B_PVDONE + 0));
+          mma_commit_w(bar(L::B_PVDONE + 0));
           if (!last) {
             // S0(n+1) overwrites the TMEM columns PV0(n) reads P0 from; the
             // tensor pipe executes this thread's MMAs in issue order, so it is
             // issued right behind PV0(n) without waiting for its completion.
-            if (!(ok = ra_wait(bar(L::B_KFULL + ks1), ((n + 1) / L::KS) & 1, abort_flag))) break;
+            if (!(ok = ra_wait_warp(bar(L::B_KFULL + ks1), ((n + 1) / L::KS) & 1, abort_flag))) break;
             issue_s(0, ks1);
-            mma_commit(bar(L::B_SFULL + 0));
+            mma_commit_w(bar(L::B_SFULL + 0));
           }
           // query tile 1
-          if (!(ok = ra_wait(bar(L::B_PFULL + 1), ph, abort_flag))) break;
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 1), ph, abort_flag))) break;
           tc_fence_after();
           issue_pv(1, vs, n > 0);
-          mma_commit(bar(L::B_PVDONE + 1));
-          mma_commit(bar(L::B_VEMPTY + vs));
+          mma_commit_w(bar(L::B_PVDONE + 1));
+          mma_commit_w(bar(L::B_VEMPTY + vs));
           if (!last) {
             issue_s(1, ks1);
-            mma_commit(bar(L::B_SFULL + 1));
-            mma_commit(bar(L::B_KEMPTY + ks1));
+            mma_commit_w(bar(L::B_SFULL + 1));
+            mma_commit_w(bar(L::B_KEMPTY + ks1));
           }
           if (last) break;
         }
       }
       // Every MMA and commit issued above must complete before TMEM is freed
       // and before the block's shared memory (barriers included) is released.
-      mma_commit(bar(L::B_DRAIN));
+      mma_commit_w(bar(L::B_DRAIN));
       ra_wait_drain(bar(L::B_DRAIN), 0);
     }
     __syncwarp();
