@@ -35,8 +35,10 @@ sys.path.insert(0, ROOT)
 METRIC = "attention TFLOP/s (fwd, fwd+bwd) at 32K-1M tokens; % of B200 dense BF16 peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SRC = os.path.join(ROOT, "long_context_exact_ordered_b200", "csrc", "ra_bwd_sm100.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ra_bwd_sm100_causal16k.md")
+# The backward kernel's sources; the committed DRAM capture is void once any of them changes.
+KERNEL_SRCS = [os.path.join(ROOT, "long_context_exact_ordered_b200", "csrc", f)
+               for f in ("ra_bwd_sm100.cuh", "ra_common.cuh", "ptx.cuh")]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ra_bwd_sm100_causal128k_dram.md")
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -134,6 +136,13 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
 
 
+def kernel_sources_sha256() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SRCS:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()
+
+
 def traffic_per_launch():
     """dram bytes per launch of the backward kernel from the committed ncu summary,
     or None when the kernel source changed since those counters were taken."""
@@ -142,10 +151,10 @@ def traffic_per_launch():
     except OSError:
         return None, None
     m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    s = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    s = re.search(r"kernel_sources_sha256:\s*([0-9a-f]+)", text)
     if not m or not s:
         return None, None
-    cur = hashlib.sha256(open(KERNEL_SRC, "rb").read()).hexdigest()
+    cur = kernel_sources_sha256()
     if cur != s.group(1):
         return None, "kernel changed since the ncu capture"
     return float(m.group(1)), None

@@ -61,16 +61,18 @@ def test_reference_arm_is_silent_on_other_ranks():
     assert r.stdout.strip() == ""
 
 
-def test_traffic_summary_is_tied_to_kernel_source(tmp_path, monkeypatch):
-    src = tmp_path / "k.cuh"
-    src.write_text("kernel v1")
+def test_traffic_summary_is_tied_to_kernel_sources(tmp_path, monkeypatch):
     import hashlib
 
-    sha = hashlib.sha256(b"kernel v1").hexdigest()
+    srcs = [tmp_path / "a.cuh", tmp_path / "b.cuh"]
+    srcs[0].write_text("kernel v1")
+    srcs[1].write_text("helpers v1")
+    sha = hashlib.sha256(b"kernel v1" + b"helpers v1").hexdigest()
     summ = tmp_path / "t.md"
-    summ.write_text("traffic_bytes_per_launch: 1.5e6\nkernel_source_sha256: %s\n" % sha)
-    monkeypatch.setattr(bench, "KERNEL_SRC", str(src))
+    summ.write_text("traffic_bytes_per_launch: 1.5e6\nkernel_sources_sha256: %s\n" % sha)
+    monkeypatch.setattr(bench, "KERNEL_SRCS", [str(x) for x in srcs])
     monkeypatch.setattr(bench, "TRAFFIC_FILE", str(summ))
     assert bench.traffic_per_launch()[0] == 1.5e6
-    src.write_text("kernel v2")
+    srcs[1].write_text("helpers v2")          # a change in any source voids the capture
     assert bench.traffic_per_launch()[0] is None
+
