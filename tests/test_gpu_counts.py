@@ -54,6 +54,9 @@ CASES = [
     (128, 1024, 1, None, None, "neginf", None),
     (64, 1024, 4, 1, "packed", "neginf", None),
     (64, 2048, 8, 5, None, None, [7, 6, 5, 4, 3, 2, 1, 0]),
+    (128, 1000, 2, 1, "packed", "neginf", None),        # ragged last tile (1000 = 7 * 128 + 104)
+    (128, 1000, 4, None, None, None, [1, 3, 0, 2]),
+    (64, 1000, 4, 3, "packed", None, None),
 ]
 
 
