@@ -283,29 +283,25 @@ def run_ours(args):
 
 
 def run_e2e(args, w, inp, kw, dev, n_vis, world):
-    """Same metric through the public API with host buffers: pinned H2D of q,k,v,dO,
-    forward + backward, D2H of o, lse, dq, dk, dv, every step."""
+    """Same metric through the public host-buffer API (HostStep -> ra_train_step_host):
+    every step copies q, k, v, dO from pinned host memory and o, lse, dq, dk, dv
+    back, overlapped with the kernels by head groups."""
     import torch
 
     import long_context_exact_ordered_b200 as ra
 
     names = ("q", "k", "v", "do")
     host = {n: inp[n].cpu().pin_memory() for n in names}
-    dbuf = {n: torch.empty_like(inp[n]) for n in names}
     outs_h = [torch.empty(inp["q"].shape, dtype=inp["q"].dtype, pin_memory=True) for _ in range(4)]
     lse_h = torch.empty((w.B, w.H, w.S), dtype=torch.float32, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in outs_h) + lse_h.numel() * 4
+    step = ra.HostStep(w.B, w.S, w.H, w.D, dtype=inp["q"].dtype, device=dev, has_bias=inp["bias"] is not None,
+                       has_segments=inp["seg"] is not None, **kw)
 
     def one():
-        for n in names:
-            dbuf[n].copy_(host[n], non_blocking=True)
-        o, lse = ra.ringattention(dbuf["q"], dbuf["k"], dbuf["v"], inp["bias"], inp["seg"], **kw)
-        dq, dk, dv = ra.ringattention_backward(dbuf["q"], dbuf["k"], dbuf["v"], o, lse, dbuf["do"], inp["bias"],
-                                               inp["seg"], **kw)
-        for hsrc, dsrc in zip(outs_h, (o, dq, dk, dv)):
-            hsrc.copy_(dsrc, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        step(host["q"], host["k"], host["v"], host["do"], outs_h[0], lse_h, outs_h[1], outs_h[2], outs_h[3],
+             attention_bias=inp["bias"], segment_ids=inp["seg"])
 
     one()
     torch.cuda.synchronize()
@@ -319,8 +315,12 @@ def run_e2e(args, w, inp, kw, dev, n_vis, world):
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     val = aggregate(14.0 * w.D * n_vis * n, ms / 1e3, world) / 1e12
+    hpg = step.hpg
+    del step
     return {"value": round(val, 2), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": n, "ms_per_step": round(ms / n, 3)}
+            "steps": n, "ms_per_step": round(ms / n, 3),
+            "api": "HostStep / ra_train_step_host: host-buffer fwd+bwd, copies overlapped by head groups",
+            "heads_per_group": hpg}
 
 
 # ---------------------------------------------------------------- CPU oracle (baseline / reference arm)

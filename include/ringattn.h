@@ -189,6 +189,44 @@ int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* 
 int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* attention_bias,
                       const ra_tensor* segment_ids, const ra_params* p, ra_tensor* o, ra_tensor* lse, void* stream);
 
+/* Tensors of one training step whose inputs and outputs live in HOST memory
+ * (ra_train_step_host).  Host tensors should be page-locked (cudaHostAlloc /
+ * pinned torch tensors) for the copies to overlap with the kernels.  Every
+ * tensor here must be contiguous: [B,S,H,D] row-major for q .. dv and their
+ * device twins, [B,H,S] for lse. */
+typedef struct {
+  ra_tensor q, k, v, d_o;                 /* HOST inputs, [B,S,H,D], bf16 or fp32 */
+  ra_tensor o, lse, dq, dk, dv;           /* HOST outputs: o, dq, dk, dv like q; lse fp32 [B,H,S] */
+  ra_tensor dev_q, dev_k, dev_v, dev_do;  /* DEVICE staging, same shapes and dtypes as the host twins */
+  ra_tensor dev_o, dev_lse, dev_dq, dev_dk, dev_dv;
+} ra_host_step;
+
+/* Forward and backward of one training step with every input and output in
+ * host memory: the end-to-end call of a training loop that keeps its
+ * tensors on the host.  The definition computes every (batch, head) pair
+ * independently, so the step is cut into groups of heads_per_group heads
+ * and pipelined over
+ * three streams: the host->device copy of group g+1 (h2d_stream) runs while
+ * the kernels of group g run (compute_stream), and the device->host copy of
+ * group g-1's results (d2h_stream) runs beside both.  Per group the work is
+ * exactly ra_forward followed by ra_backward on that group's heads, so the
+ * results equal those two calls on the whole tensors.
+ *  t: the tensors (see ra_host_step); dq, dk, dv take the dtype of q.
+ *  attention_bias / segment_ids: NULL or DEVICE tensors as in ra_forward.
+ *  heads_per_group: >= 1 and divides H.
+ *  workspace: DEVICE, at least ra_workspace_size(1, q', p, ...) bytes for q'
+ *  = q with H replaced by heads_per_group (reused by every group).
+ *  Streams may coincide (then nothing overlaps).  The call is asynchronous;
+ *  compute_stream is made to wait for the last device->host copy, so
+ *  synchronizing compute_stream covers the whole step.  Calls using the
+ *  same buffers are serialized through compute_stream.  The library creates
+ *  and releases CUDA events inside the call and allocates no memory.
+ *  Returns the first error of any part; outputs are then unspecified, and
+ *  part of the step may already have been queued. */
+int ra_train_step_host(const ra_host_step* t, const ra_tensor* attention_bias, const ra_tensor* segment_ids,
+                       const ra_params* p, int64_t heads_per_group, void* workspace, size_t workspace_bytes,
+                       void* compute_stream, void* h2d_stream, void* d2h_stream);
+
 /* Synchronizes `stream`, returns the device status word of the current
  * device (RA_OK or RA_ERR_DEVICE_TIMEOUT) and clears it.  RA_ERR_CUDA if
  * the synchronization itself failed. */

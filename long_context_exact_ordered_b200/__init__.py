@@ -5,6 +5,7 @@ ABI, include/ringattn.h); this package only marshals torch tensors into it.
 """
 
 from .api import (  # noqa: F401
+    HostStep,
     RingAttentionFunction,
     count_visible_pairs,
     device_status,
@@ -25,5 +26,5 @@ from ._lib import RingAttnError, load  # noqa: F401
 __all__ = [
     "ringattention", "ringattention_backward", "ringattention_static", "ring_step", "init_state", "finalize", "lse_merge",
     "device_status", "selftest_timeout", "count_visible_pairs", "ring_schedule", "workspace_size", "RingAttentionFunction", "visible_count_probe",
-    "RingAttnError", "load",
+    "HostStep", "RingAttnError", "load",
 ]

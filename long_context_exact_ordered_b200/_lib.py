@@ -47,6 +47,11 @@ class RaParams(ctypes.Structure):
     ]
 
 
+class RaHostStep(ctypes.Structure):
+    _fields_ = [(n, RaTensor) for n in ("q", "k", "v", "d_o", "o", "lse", "dq", "dk", "dv", "dev_q", "dev_k", "dev_v",
+                                         "dev_do", "dev_o", "dev_lse", "dev_dq", "dev_dk", "dev_dv")]
+
+
 _T = ctypes.POINTER(RaTensor)
 _P = ctypes.POINTER(RaParams)
 _vp = ctypes.c_void_p
@@ -59,6 +64,8 @@ SIGNATURES = {
     "ra_step": (ctypes.c_int, [_T, _T, _T, ctypes.c_int64, ctypes.c_int64, _T, _T, _T, _P, _T, _T, _T, _vp]),
     "ra_finalize": (ctypes.c_int, [_T, _T, _T, _T, _T, _vp]),
     "ra_lse_merge": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, _vp]),
+    "ra_train_step_host": (ctypes.c_int, [ctypes.POINTER(RaHostStep), _T, _T, _P, ctypes.c_int64, _vp,
+                                          ctypes.c_size_t, _vp, _vp, _vp]),
     "ra_get_device_status": (ctypes.c_int, [_vp]),
     "ra_selftest_timeout": (ctypes.c_int, [ctypes.c_int64, _vp]),
     "ra_strerror": (ctypes.c_char_p, [ctypes.c_int]),

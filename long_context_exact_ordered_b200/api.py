@@ -15,7 +15,7 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import RA_BF16, RA_F32, RA_I32, RA_MAX_RING, RaParams, RaTensor, check, load
+from ._lib import RA_BF16, RA_F32, RA_I32, RA_MAX_RING, RaHostStep, RaParams, RaTensor, check, load
 
 _DT = {torch.float32: RA_F32, torch.bfloat16: RA_BF16, torch.int32: RA_I32}
 
@@ -301,3 +301,67 @@ def visible_count_probe(fwd_row_counts=None, bwd_col_counts=None):
     finally:
         _lib.swap(prev)
         dbg.ra_debug_set_counts(None, None)
+
+
+class HostStep:
+    """One training step (forward + backward) whose inputs and outputs live in
+    host memory, through ``ra_train_step_host``: the heads are processed in
+    groups, and each group's host->device copy, kernels and device->host copy
+    run on three streams so the copies overlap the kernels.
+
+    The object owns the device staging buffers, the workspace and two copy
+    streams, sized once for [B, S, H, D] tensors of ``dtype``; call it once
+    per step with pinned host tensors.  The kernels run on the caller's
+    current stream, which is made to wait for the last copy back."""
+
+    def __init__(self, B, S, H, D, dtype=torch.bfloat16, heads_per_group=None, device=None, has_bias=False,
+                 has_segments=False, query_chunk_size=512, key_chunk_size=512, causal_block_size=None,
+                 ring_size=1, ring_order=None):
+        device = torch.device("cuda") if device is None else torch.device(device)
+        if heads_per_group is None:                  # about eight groups: one copy in, one out exposed per step
+            heads_per_group = max(1, H // 8)
+            while H % heads_per_group:
+                heads_per_group -= 1
+        self.shape, self.dtype, self.hpg = (B, S, H, D), dtype, int(heads_per_group)
+        self.params = _params(S, query_chunk_size, key_chunk_size, causal_block_size, ring_size, ring_order)
+        mk = lambda: torch.empty((B, S, H, D), dtype=dtype, device=device)
+        self.dev = {n: mk() for n in ("q", "k", "v", "do", "o", "dq", "dk", "dv")}
+        self.dev["lse"] = torch.empty((B, H, S), dtype=torch.float32, device=device)
+        probe = torch.empty((B, S, self.hpg, D), dtype=dtype, device="meta")
+        n = load().ra_workspace_size(1, ctypes.byref(_tensor_meta(probe)), ctypes.byref(self.params),
+                                     int(has_bias), int(has_segments))
+        self.workspace = _workspace(n, device)
+        self.h2d = torch.cuda.Stream(device)
+        self.d2h = torch.cuda.Stream(device)
+
+    def __call__(self, q, k, v, do, o, lse, dq, dk, dv, attention_bias=None, segment_ids=None):
+        """q, k, v, do: host [B,S,H,D]; o, dq, dk, dv: host outputs like q; lse: host fp32 [B,H,S].
+        attention_bias / segment_ids: device tensors or None."""
+        for x in (q, k, v, do, o, lse, dq, dk, dv):
+            if x.is_cuda:
+                raise ValueError("HostStep takes host tensors (pinned for overlap)")
+        t = RaHostStep()
+        for name, x in (("q", q), ("k", k), ("v", v), ("d_o", do), ("o", o), ("lse", lse), ("dq", dq), ("dk", dk),
+                        ("dv", dv)):
+            setattr(t, name, _tensor(x))
+        for name, key in (("dev_q", "q"), ("dev_k", "k"), ("dev_v", "v"), ("dev_do", "do"), ("dev_o", "o"),
+                          ("dev_lse", "lse"), ("dev_dq", "dq"), ("dev_dk", "dk"), ("dev_dv", "dv")):
+            setattr(t, name, _tensor(self.dev[key]))
+        ws = self.workspace
+        code = load().ra_train_step_host(ctypes.byref(t), _ref(_tensor(attention_bias)), _ref(_tensor(segment_ids)),
+                                         ctypes.byref(self.params), self.hpg, 0 if ws is None else ws.data_ptr(),
+                                         0 if ws is None else ws.numel(), _stream(), self.h2d.cuda_stream,
+                                         self.d2h.cuda_stream)
+        check(code, "ra_train_step_host")
+
+
+def _tensor_meta(t: torch.Tensor) -> RaTensor:
+    """Shape-only descriptor (no data) for size queries."""
+    r = RaTensor()
+    r.data = 0
+    r.dtype = _DT[t.dtype]
+    r.ndim = t.dim()
+    for i in range(t.dim()):
+        r.shape[i] = t.shape[i]
+        r.stride[i] = t.stride(i)
+    return r

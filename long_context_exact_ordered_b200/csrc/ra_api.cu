@@ -747,6 +747,134 @@ int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v
   return ra_forward(q, k, v, attention_bias, segment_ids, p, o, lse, scratch, RA_STATIC_SCRATCH_BYTES, stream);
 }
 
+namespace {
+
+bool contiguous_bshd(const ra_tensor* t) {
+  return t && t->ndim == 4 && t->stride[3] == 1 && t->stride[2] == t->shape[3] &&
+         t->stride[1] == t->shape[2] * t->shape[3] && t->stride[0] == t->shape[1] * t->stride[1];
+}
+bool contiguous_bhs(const ra_tensor* t) {
+  return t && t->ndim == 3 && t->stride[2] == 1 && t->stride[1] == t->shape[2] &&
+         t->stride[0] == t->shape[1] * t->shape[2];
+}
+bool same_shape(const ra_tensor* a, const ra_tensor* b) {
+  if (a->ndim != b->ndim || a->dtype != b->dtype) return false;
+  for (int i = 0; i < a->ndim; ++i)
+    if (a->shape[i] != b->shape[i]) return false;
+  return true;
+}
+size_t elem_bytes(int dt) { return dt == RA_BF16 ? 2 : 4; }
+
+// The heads [h0, h0 + hg) of a contiguous [B,S,H,D] tensor, as a strided view.
+ra_tensor head_view(const ra_tensor& t, int64_t h0, int64_t hg) {
+  ra_tensor v = t;
+  v.data = static_cast<char*>(t.data) + h0 * t.shape[3] * elem_bytes(t.dtype);
+  v.shape[2] = hg;
+  return v;
+}
+// The heads [h0, h0 + hg) of a contiguous [B,H,S] tensor.
+ra_tensor head_view_bhs(const ra_tensor& t, int64_t h0, int64_t hg) {
+  ra_tensor v = t;
+  v.data = static_cast<char*>(t.data) + h0 * t.shape[2] * 4;
+  v.shape[1] = hg;
+  return v;
+}
+// Copy heads [h0, h0 + hg) of a contiguous [B,S,H,D] tensor: B*S rows of
+// hg*D elements, pitch H*D elements.
+cudaError_t copy_heads(const ra_tensor& dst, const ra_tensor& src, int64_t h0, int64_t hg, cudaMemcpyKind kind,
+                       cudaStream_t st) {
+  const size_t e = elem_bytes(src.dtype), D = (size_t)src.shape[3], H = (size_t)src.shape[2];
+  const size_t off = (size_t)h0 * D * e, pitch = H * D * e;
+  return cudaMemcpy2DAsync(static_cast<char*>(dst.data) + off, pitch, static_cast<const char*>(src.data) + off,
+                           pitch, (size_t)hg * D * e, (size_t)(src.shape[0] * src.shape[1]), kind, st);
+}
+// Heads [h0, h0 + hg) of a contiguous fp32 [B,H,S] tensor: B rows of hg*S floats.
+cudaError_t copy_heads_bhs(const ra_tensor& dst, const ra_tensor& src, int64_t h0, int64_t hg, cudaMemcpyKind kind,
+                           cudaStream_t st) {
+  const size_t S = (size_t)src.shape[2], H = (size_t)src.shape[1];
+  const size_t off = (size_t)h0 * S * 4, pitch = H * S * 4;
+  return cudaMemcpy2DAsync(static_cast<char*>(dst.data) + off, pitch, static_cast<const char*>(src.data) + off,
+                           pitch, (size_t)hg * S * 4, (size_t)src.shape[0], kind, st);
+}
+
+struct EventPool {   // events of one call, released on every return path
+  std::vector<cudaEvent_t> ev;
+  ~EventPool() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);   // pending events are released once they complete
+  }
+  cudaEvent_t make() {
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    ev.push_back(e);
+    return e;
+  }
+};
+
+}  // namespace
+
+int ra_train_step_host(const ra_host_step* t, const ra_tensor* attention_bias, const ra_tensor* segment_ids,
+                       const ra_params* p, int64_t heads_per_group, void* workspace, size_t workspace_bytes,
+                       void* compute_stream, void* h2d_stream, void* d2h_stream) {
+  if (!t || !p) return RA_ERR_NULL;
+  const ra_tensor* bshd[] = {&t->q, &t->k, &t->v, &t->d_o, &t->o, &t->dq, &t->dk, &t->dv,
+                             &t->dev_q, &t->dev_k, &t->dev_v, &t->dev_do, &t->dev_o, &t->dev_dq, &t->dev_dk,
+                             &t->dev_dv};
+  for (const ra_tensor* x : bshd)
+    if (!x->data) return RA_ERR_NULL;
+  if (!t->lse.data || !t->dev_lse.data) return RA_ERR_NULL;
+  for (const ra_tensor* x : bshd)
+    if (x->ndim != 4) return RA_ERR_SHAPE;
+  for (const ra_tensor* x : bshd)
+    if (!same_shape(x, &t->q)) return x->dtype != t->q.dtype ? RA_ERR_DTYPE : RA_ERR_SHAPE;
+  for (const ra_tensor* x : bshd)
+    if (!contiguous_bshd(x)) return RA_ERR_STRIDE;
+  const int64_t B = t->q.shape[0], S = t->q.shape[1], H = t->q.shape[2];
+  for (const ra_tensor* x : {&t->lse, &t->dev_lse}) {
+    if (x->ndim != 3 || x->dtype != RA_F32) return x->ndim != 3 ? RA_ERR_SHAPE : RA_ERR_DTYPE;
+    if (x->shape[0] != B || x->shape[1] != H || x->shape[2] != S) return RA_ERR_SHAPE;
+    if (!contiguous_bhs(x)) return RA_ERR_STRIDE;
+  }
+  if (heads_per_group < 1 || H % heads_per_group) return RA_ERR_DIVISIBILITY;
+  if (B * S * H == 0) return RA_OK;
+  cudaStream_t sc = static_cast<cudaStream_t>(compute_stream), si = static_cast<cudaStream_t>(h2d_stream),
+               so = static_cast<cudaStream_t>(d2h_stream);
+  EventPool pool;
+  // The copies of this step start after everything queued before it on compute_stream.
+  cudaEvent_t start = pool.make();
+  if (!start || cudaEventRecord(start, sc) != cudaSuccess) return RA_ERR_CUDA;
+  if (cudaStreamWaitEvent(si, start, 0) != cudaSuccess || cudaStreamWaitEvent(so, start, 0) != cudaSuccess)
+    return RA_ERR_CUDA;
+  const int64_t hg = heads_per_group;
+  for (int64_t h0 = 0; h0 < H; h0 += hg) {
+    const ra_tensor* in_h[] = {&t->q, &t->k, &t->v, &t->d_o};
+    const ra_tensor* in_d[] = {&t->dev_q, &t->dev_k, &t->dev_v, &t->dev_do};
+    for (int i = 0; i < 4; ++i)
+      if (copy_heads(*in_d[i], *in_h[i], h0, hg, cudaMemcpyHostToDevice, si) != cudaSuccess) return RA_ERR_CUDA;
+    cudaEvent_t landed = pool.make(), done = pool.make();
+    if (!landed || !done) return RA_ERR_CUDA;
+    if (cudaEventRecord(landed, si) != cudaSuccess || cudaStreamWaitEvent(sc, landed, 0) != cudaSuccess)
+      return RA_ERR_CUDA;
+    ra_tensor q = head_view(t->dev_q, h0, hg), k = head_view(t->dev_k, h0, hg), v = head_view(t->dev_v, h0, hg),
+              d_o = head_view(t->dev_do, h0, hg), o = head_view(t->dev_o, h0, hg),
+              dq = head_view(t->dev_dq, h0, hg), dk = head_view(t->dev_dk, h0, hg),
+              dv = head_view(t->dev_dv, h0, hg), lse = head_view_bhs(t->dev_lse, h0, hg);
+    RA_TRY(ra_forward(&q, &k, &v, attention_bias, segment_ids, p, &o, &lse, workspace, workspace_bytes, sc));
+    RA_TRY(ra_backward(&q, &k, &v, &o, &d_o, &lse, attention_bias, segment_ids, p, &dq, &dk, &dv, workspace,
+                       workspace_bytes, sc));
+    if (cudaEventRecord(done, sc) != cudaSuccess || cudaStreamWaitEvent(so, done, 0) != cudaSuccess)
+      return RA_ERR_CUDA;
+    const ra_tensor* out_d[] = {&t->dev_o, &t->dev_dq, &t->dev_dk, &t->dev_dv};
+    const ra_tensor* out_h[] = {&t->o, &t->dq, &t->dk, &t->dv};
+    for (int i = 0; i < 4; ++i)
+      if (copy_heads(*out_h[i], *out_d[i], h0, hg, cudaMemcpyDeviceToHost, so) != cudaSuccess) return RA_ERR_CUDA;
+    if (copy_heads_bhs(t->lse, t->dev_lse, h0, hg, cudaMemcpyDeviceToHost, so) != cudaSuccess) return RA_ERR_CUDA;
+  }
+  cudaEvent_t fin = pool.make();
+  if (!fin || cudaEventRecord(fin, so) != cudaSuccess || cudaStreamWaitEvent(sc, fin, 0) != cudaSuccess)
+    return RA_ERR_CUDA;
+  return RA_OK;
+}
+
 int ra_selftest_timeout(int64_t budget_cycles, void* stream) {
   if (budget_cycles < 1000 || budget_cycles > 1000000000ll) return RA_ERR_UNSUPPORTED;
   int* ptr = nullptr;

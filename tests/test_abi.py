@@ -209,3 +209,43 @@ def test_selftest_timeout_rejects_bad_budgets_on_host():
     lib = _lib.load()
     assert lib.ra_selftest_timeout(10, None) == 6          # below the allowed range
     assert lib.ra_selftest_timeout(10 ** 10, None) == 6    # above it
+
+
+def _host_step(B=1, S=256, H=4, D=64, dtype=_lib.RA_BF16):
+    t = _lib.RaHostStep()
+    for name in ("q", "k", "v", "d_o", "o", "dq", "dk", "dv", "dev_q", "dev_k", "dev_v", "dev_do", "dev_o", "dev_dq",
+                 "dev_dk", "dev_dv"):
+        setattr(t, name, T([B, S, H, D], dtype))
+    t.lse = T([B, H, S], _lib.RA_F32)
+    t.dev_lse = T([B, H, S], _lib.RA_F32)
+    return t
+
+
+def test_train_step_host_argument_errors():
+    """ra_train_step_host rejects bad arguments before any stream, event or copy."""
+    lib = _lib.load()
+    p = P()
+
+    def call(t, hpg=2):
+        return lib.ra_train_step_host(ctypes.byref(t) if t is not None else None, None, None, ctypes.byref(p), hpg,
+                                      None, 0, None, None, None)
+
+    assert call(None) == 1                                                  # RA_ERR_NULL
+    t = _host_step()
+    t.dev_dk.data = 0
+    assert call(t) == 1                                                     # a missing buffer
+    t = _host_step()
+    t.dq = T([1, 256, 4, 64], _lib.RA_F32)
+    assert call(t) == 2                                                     # gradients take q's dtype
+    t = _host_step()
+    t.dev_v = T([1, 128, 4, 64])
+    assert call(t) == 3                                                     # device twin of another shape
+    t = _host_step()
+    t.k = T([1, 256, 4, 64], strides=[256 * 4 * 64, 4 * 64, 64 * 2, 1])   # heads not packed
+    assert call(t) == 4                                                     # RA_ERR_STRIDE: not contiguous
+    t = _host_step()
+    t.lse = T([1, 256, 4], _lib.RA_F32)
+    assert call(t) == 3                                                     # lse is [B, H, S]
+    t = _host_step()
+    assert call(t, hpg=3) == 5                                              # 3 does not divide H = 4
+    assert call(t, hpg=0) == 5
