@@ -22,7 +22,7 @@ DEBUG_HEADER = os.path.join(ROOT, "include", "ringattn_debug.h")
 def declared_functions(header=HEADER):
     text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(ra_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(ra_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_every_declared_symbol_is_exported():
