@@ -25,7 +25,7 @@ extern "C" {
 
 /* Sets (or, with NULL, clears) the count buffers used by every later
  * ra_forward / ra_backward call of this process that takes the tensor-core
- * path (bf16 q/k/v; the backward with D = 128).
+ * path (bf16 q/k/v, D = 64 or 128).
  *  - fwd_row_counts: DEVICE int32 [B, H, S], contiguous: for each query row,
  *    the number of keys the forward kernel let into its softmax.  Every row
  *    below S is overwritten by each forward call.

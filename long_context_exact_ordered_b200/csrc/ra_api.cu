@@ -323,10 +323,11 @@ int launch_fwd_simt(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, 
   return last_cuda();
 }
 
+template <int D>
 int launch_bwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* d_o,
                      const MaskArgs& mk, const RingDesc& rd, const int4* meta, const WsLayout& w, char* ws,
                      ra_tensor* dk, ra_tensor* dv, cudaStream_t st) {
-  using L = BwdLayout;
+  using L = BwdLayout<D>;
   CUtensorMap tq, tk, tv, tdo, tdq;
   RA_TRY(make_tmap_bshd(&tq, q, L::QT));
   RA_TRY(make_tmap_bshd(&tk, k, kTile));
@@ -366,10 +367,10 @@ int launch_bwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v,
 #endif
   const int64_t grid = (int64_t)rd.ntiles * prm.B * prm.H;
   if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(ra_bwd_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
+  if (cudaFuncSetAttribute(ra_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
       cudaSuccess)
     return RA_ERR_CUDA;
-  ra_bwd_sm100_kernel<<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, tdq, prm);
+  ra_bwd_sm100_kernel<D><<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, tdq, prm);
   return last_cuda();
 }
 
@@ -513,7 +514,7 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   const MaskArgs mk = mask_args(attention_bias, segment_ids);
   char* ws = static_cast<char*>(workspace);
   int4* meta = need_meta ? reinterpret_cast<int4*>(ws + w.meta) : nullptr;
-  const bool tc_path = dt == RA_BF16 && D == 128;   // tensor-core backward; else CUDA cores
+  const bool tc_path = dt == RA_BF16;   // tensor-core backward (D = 64 or 128); fp32 inputs on CUDA cores
   if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
   {
     BwdPreArgs pa;
@@ -535,7 +536,8 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   const ProfScope prof(p, st);
   if (tc_path) {
     prof.begin();
-    const int rc = launch_bwd_sm100(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st);
+    const int rc = D == 64 ? launch_bwd_sm100<64>(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st)
+                           : launch_bwd_sm100<128>(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st);
     prof.end();
     RA_TRY(rc);
     DqConvertArgs ca{(int)B, (int)S, (int)H, (int)D, reinterpret_cast<const float*>(ws + w.dqacc),
@@ -568,8 +570,7 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   a.out_bf16 = dq->dtype == RA_BF16;
   prof.begin();
   int rc;
-  if (dt == RA_BF16) rc = launch_bwd_simt<64, __nv_bfloat16>(a, S, st);
-  else rc = D == 64 ? launch_bwd_simt<64, float>(a, S, st) : launch_bwd_simt<128, float>(a, S, st);
+  rc = D == 64 ? launch_bwd_simt<64, float>(a, S, st) : launch_bwd_simt<128, float>(a, S, st);   // fp32 inputs
   prof.end();
   return rc;
 }

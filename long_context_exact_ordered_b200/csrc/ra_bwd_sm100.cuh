@@ -1,4 +1,4 @@
-// sm_100a backward (bf16 in, fp32 accumulate, head_dim 128): gradients of
+// sm_100a backward (bf16 in, fp32 accumulate, head_dim 64 or 128): gradients of
 // blockwise exact attention, recomputing probabilities from the saved
 // log-sum-exp (the recompute policy "nothing_saveable" of page
 // "RingAttention核心功能全解析", 核心API调用).
@@ -23,16 +23,16 @@
 // warps 4-7 and 12-15 "softmax" (thread = key row; the two warpgroups take
 // query columns 0-31 and 32-63 of each tile: P^T, dS^T, then dK resp. dV in
 // the epilogue), warps 8-11 dQ readout (thread = head-dim lane d of dQ^T).
-// TMEM (512 columns): two 128-column slots, then dK [256,384), dV [384,512).
+// TMEM (512 columns): two 128-column slots, then dK [256,256+D), dV [256+D,256+2D).
 // Query tile n uses slot n % 2: S^T -> [0,64), dP^T -> [64,128); the softmax
 // group overwrites [0,32) with P^T and [32,64) with dS^T (bf16), and dQ^T(n)
 // lands in [64,128) once dP^T has been read.  A slot is reused two tiles
 // later, after the readout group has taken dQ^T out of it.
 //
 // Overlap: with two slots the "head" products of tile n+1 (S^T, dP^T) are
-// computed while the softmax groups work on tile n, and the issuing thread
-// feeds the tensor core whichever is ready first: the oldest tile's tail
-// (dV, dK, dQ^T) or the next head (slot and query stage free).
+// computed while the softmax groups work on tile n; the issue order is given
+// at the MMA issuer below.  At D = 64, dQ^T keeps M = 128 by reading a zero
+// block as the upper half of K^T, so only its first 64 rows are read out.
 #pragma once
 
 #include <cuda.h>
@@ -44,12 +44,14 @@
 
 namespace ra {
 
+template <int D_>
 struct BwdLayout {
-  static constexpr int D = 128;
+  static constexpr int D = D_;                    // 64 or 128
+  static constexpr int KCH = D / 64;              // 128-byte swizzle chunks along D
   static constexpr int QT = kQTileBwd;            // 64 query rows per tile
-  static constexpr int KV_BYTES = kTile * D * 2;  // 32 KB
+  static constexpr int KV_BYTES = kTile * D * 2;  // 32 KB at D = 128
   static constexpr int KV_CHUNK = kTile * 128;    // 16 KB box: 128 rows x 128 B
-  static constexpr int Q_BYTES = QT * D * 2;      // 16 KB
+  static constexpr int Q_BYTES = QT * D * 2;      // 16 KB at D = 128
   static constexpr int Q_CHUNK = QT * 128;        // 8 KB box: 64 rows x 128 B
   static constexpr int DS_BYTES = kTile * QT * 2; // 16 KB: 128 keys x 64 queries bf16
   static constexpr int NS = 3;                    // query-side stages (two tiles in flight + one loading)
@@ -59,10 +61,15 @@ struct BwdLayout {
   static constexpr int OFF_Q = OFF_V + KV_BYTES;
   static constexpr int OFF_DO = OFF_Q + NS * Q_BYTES;
   static constexpr int OFF_DS = OFF_DO + NS * Q_BYTES;
-  static constexpr int OFF_LD = OFF_DS + NSLOT * DS_BYTES;   // per stage: lse2[64], delta[64]
+  // dQ^T = K^T dS^T is an M = 128 product along D.  At D = 64 its second
+  // 64-row half of A reads this zero block, so rows 64..127 of dQ^T are 0.
+  static constexpr int OFF_ZERO = OFF_DS + NSLOT * DS_BYTES;
+  static constexpr int ZERO_BYTES = D == 64 ? KV_CHUNK : 0;
+  static constexpr uint32_t LBO_DQ = D == 128 ? KV_CHUNK : OFF_ZERO - OFF_K;   // distance between the D halves
+  static constexpr int OFF_LD = OFF_ZERO + ZERO_BYTES;       // per stage: lse2[64], delta[64]
   static constexpr int LD_BYTES = 2 * QT * 4;
   static constexpr int OFF_DQS = OFF_LD + NS * LD_BYTES;    // dQ staging [64][D] fp32
-  static constexpr int DQS_BYTES = QT * D * 4;               // 32 KB
+  static constexpr int DQS_BYTES = QT * D * 4;               // 32 KB at D = 128
   static constexpr int OFF_BAR = OFF_DQS + DQS_BYTES;
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1;                  // [NS] query stage loaded
@@ -82,10 +89,12 @@ struct BwdLayout {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t SLOT_COLS = 128;
   static constexpr uint32_t SLOT_ST = 0, SLOT_DPT = 64, SLOT_PT = 0, SLOT_DST = 32, SLOT_DQT = 64;
-  static constexpr uint32_t COL_DK = 256, COL_DV = 384;
+  static constexpr uint32_t COL_DK = 256, COL_DV = 256 + D;
   static constexpr int THREADS = 512;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(OFF_DQS % 128 == 0, "bulk reduce source alignment");
+  static_assert(OFF_ZERO % 1024 == 0 && LBO_DQ % 16 == 0 && (LBO_DQ >> 4) < (1u << 14), "dQ^T operand layout");
+  static_assert(D == 64 || D == 128, "head dim");
 };
 
 struct BwdParams {
@@ -138,12 +147,12 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
+template <int D>
 __global__ void __launch_bounds__(512, 1)
     ra_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ BwdParams p) {
-  using L = BwdLayout;
-  constexpr int D = L::D;
+  using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -183,6 +192,11 @@ __global__ void __launch_bounds__(512, 1)
     tmem_alloc(smem_u32(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
   }
+  if constexpr (L::ZERO_BYTES > 0) {
+    for (int i = threadIdx.x; i < L::ZERO_BYTES / 16; i += L::THREADS)
+      reinterpret_cast<uint4*>(gbase + L::OFF_ZERO)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();   // the tensor cores read it through the async proxy
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(512, 1)
       prefetch_tmap(&tm_v);
       prefetch_tmap(&tm_do);
       mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::KV_BYTES);
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < L::KCH; ++c) {
         tma_load_4d(sbase + L::OFF_K + c * L::KV_CHUNK, &tm_k, bar(L::B_KV), c * 64, h, (int)k0, b);
         tma_load_4d(sbase + L::OFF_V + c * L::KV_CHUNK, &tm_v, bar(L::B_KV), c * 64, h, (int)k0, b);
       }
@@ -217,7 +231,7 @@ __global__ void __launch_bounds__(512, 1)
           if (n >= L::NS && !ra_wait(bar(L::B_QE + st), ((n / L::NS) & 1) ^ 1, abort_flag)) break;
           const int q0 = q * L::QT;
           mbar_arrive_expect_tx(bar(L::B_QF + st), 2 * L::Q_BYTES + L::LD_BYTES);
-          for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < L::KCH; ++c) {
             tma_load_4d(sbase + L::OFF_Q + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_q, bar(L::B_QF + st), c * 64, h,
                         q0, b);
             tma_load_4d(sbase + L::OFF_DO + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_do, bar(L::B_QF + st), c * 64,
@@ -242,7 +256,7 @@ __global__ void __launch_bounds__(512, 1)
       // added to the start-address field (address >> 4, no carry: shared
       // memory ends below 2^18 bytes), keeping the issue loop short.
       const uint64_t ka_k = smem_desc_sw128(ka, 16, 1024), va_k = smem_desc_sw128(va, 16, 1024);
-      const uint64_t ka_mn = smem_desc_sw128(ka, L::KV_CHUNK, 1024);
+      const uint64_t ka_mn = smem_desc_sw128(ka, L::LBO_DQ, 1024);
       auto issue_sd = [&](uint32_t d_tmem, uint64_t a_desc, uint32_t b_base) {   // S^T or dP^T
         const uint64_t b_desc = smem_desc_sw128(b_base, 16, 1024);
 #pragma unroll
@@ -520,8 +534,10 @@ __global__ void __launch_bounds__(512, 1)
         }
         // staging tile [query c][d]: a warp writes 32 consecutive floats per row
         if (n > 0 && !ra_wait_warp(bar(L::B_DQSFREE), (n - 1) & 1, abort_flag)) break;
+        if (d < D) {   // at D = 64 the upper half of dQ^T is the zero padding
 #pragma unroll
-        for (int c = 0; c < 64; ++c) st_shared_f32(dqs + c * (D * 4) + d * 4, __uint_as_float(r[c]) * p.scale);
+          for (int c = 0; c < 64; ++c) st_shared_f32(dqs + c * (D * 4) + d * 4, __uint_as_float(r[c]) * p.scale);
+        }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(L::B_DQSFULL));

@@ -83,7 +83,8 @@ CASES = [
     (128, 1024, 4, 1, "packed", None, 1, 2),
     (128, 640, 5, 1, "packed", "neginf", 2, 2),
     (128, 768, 2, None, None, "neginf", 1, 2),
-    (64, 512, 2, 1, "packed", None, 1, 2),       # head_dim 64 (CUDA-core backward)
+    (64, 512, 2, 1, "packed", None, 1, 2),       # head_dim 64 (tensor cores, zero-padded dQ^T)
+    (64, 1000, 4, None, None, "neginf", 2, 2),   # head_dim 64, ragged, non-causal, masked keys
 ]
 
 

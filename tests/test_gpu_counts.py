@@ -91,7 +91,7 @@ def test_forward_counts_match_integer_mask(D, S, P, c, segments, bias, order):
     np.testing.assert_array_equal(rows.cpu().numpy().astype(np.int64), _expect(w, inp, cols=False))
 
 
-@pytest.mark.parametrize("D,S,P,c,segments,bias,order", [x for x in CASES if x[0] == 128])
+@pytest.mark.parametrize("D,S,P,c,segments,bias,order", CASES)
 def test_backward_counts_match_integer_mask(D, S, P, c, segments, bias, order):
     w, inp = make(D, S, P, c, segments, bias)
     kw = dict(query_chunk_size=w.chunk, key_chunk_size=w.chunk, causal_block_size=c, ring_size=P, ring_order=order)
