@@ -232,6 +232,16 @@ __device__ __forceinline__ void mma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint6
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// One elected lane of a converged warp (the others skip the guarded block).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(e));
+  return e != 0;
+}
 // The commit comes from the same elected lane (elect.sync is a function of
 // the active mask, which is the full warp at every call site).
 __device__ __forceinline__ void mma_commit_w(uint32_t bar) {

@@ -210,35 +210,43 @@ __global__ void __launch_bounds__(512, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_do);
-      mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::KV_BYTES);
-      for (int c = 0; c < L::KCH; ++c) {
-        tma_load_4d(sbase + L::OFF_K + c * L::KV_CHUNK, &tm_k, bar(L::B_KV), c * 64, h, (int)k0, b);
-        tma_load_4d(sbase + L::OFF_V + c * L::KV_CHUNK, &tm_v, bar(L::B_KV), c * 64, h, (int)k0, b);
+    // The whole warp runs the loop (its lanes scan 32 query tiles per
+    // metadata round trip, q_iter_next_warp); one elected lane issues copies.
+    {
+      if (elect_one()) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+        mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::KV_BYTES);
+        for (int c = 0; c < L::KCH; ++c) {
+          tma_load_4d(sbase + L::OFF_K + c * L::KV_CHUNK, &tm_k, bar(L::B_KV), c * 64, h, (int)k0, b);
+          tma_load_4d(sbase + L::OFF_V + c * L::KV_CHUNK, &tm_v, bar(L::B_KV), c * 64, h, (int)k0, b);
+        }
       }
+      __syncwarp();
       int n = 0;
       if (!dead) {
         QIter it;
         q_iter_init(it, p.rd, k0, meta_b, use_seg);
         const float* lse_row = p.lse2 + (int64_t)bh * p.s_pad;
         const float* dl_row = p.delta + (int64_t)bh * p.s_pad;
-        for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
+        for (int32_t q = q_iter_next_warp(it, p.rd); q >= 0; q = q_iter_next_warp(it, p.rd), ++n) {
           const int st = n % L::NS;
-          if (n >= L::NS && !ra_wait(bar(L::B_QE + st), ((n / L::NS) & 1) ^ 1, abort_flag)) break;
+          if (n >= L::NS && !ra_wait_warp(bar(L::B_QE + st), ((n / L::NS) & 1) ^ 1, abort_flag)) break;
           const int q0 = q * L::QT;
-          mbar_arrive_expect_tx(bar(L::B_QF + st), 2 * L::Q_BYTES + L::LD_BYTES);
-          for (int c = 0; c < L::KCH; ++c) {
-            tma_load_4d(sbase + L::OFF_Q + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_q, bar(L::B_QF + st), c * 64, h,
-                        q0, b);
-            tma_load_4d(sbase + L::OFF_DO + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_do, bar(L::B_QF + st), c * 64,
-                        h, q0, b);
+          if (elect_one()) {
+            mbar_arrive_expect_tx(bar(L::B_QF + st), 2 * L::Q_BYTES + L::LD_BYTES);
+            for (int c = 0; c < L::KCH; ++c) {
+              tma_load_4d(sbase + L::OFF_Q + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_q, bar(L::B_QF + st), c * 64, h,
+                          q0, b);
+              tma_load_4d(sbase + L::OFF_DO + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_do, bar(L::B_QF + st), c * 64,
+                          h, q0, b);
+            }
+            bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES, lse_row + q0, L::QT * 4, bar(L::B_QF + st));
+            bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES + L::QT * 4, dl_row + q0, L::QT * 4, bar(L::B_QF + st));
           }
-          bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES, lse_row + q0, L::QT * 4, bar(L::B_QF + st));
-          bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES + L::QT * 4, dl_row + q0, L::QT * 4, bar(L::B_QF + st));
+          __syncwarp();
         }
       }
       ra_wait_drain(bar(L::B_KV), 0);
@@ -283,7 +291,7 @@ __global__ void __launch_bounds__(512, 1)
       if (!dead) {
         QIter it;
         q_iter_init(it, p.rd, k0, meta_b, use_seg);
-        while (q_iter_next(it, p.rd) >= 0) ++N;
+        while (q_iter_next_warp(it, p.rd) >= 0) ++N;
       }
       // Issue order (two TMEM slots, tile n in slot n % 2):
       //   S^T(0) dP^T(0) S^T(1) dP^T(1) | tail(0) S^T(2) dP^T(2) | tail(1) S^T(3) dP^T(3) | ...
@@ -355,7 +363,7 @@ __global__ void __launch_bounds__(512, 1)
     if (!dead) {
       QIter it;
       q_iter_init(it, p.rd, k0, meta_b, use_seg);
-      for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
+      for (int32_t q = q_iter_next_warp(it, p.rd); q >= 0; q = q_iter_next_warp(it, p.rd), ++n) {
         const int st = n % L::NS, s = n & 1;
         const uint32_t slot = trow + s * L::SLOT_COLS;
         const int64_t q0 = (int64_t)q * L::QT;
@@ -511,7 +519,7 @@ __global__ void __launch_bounds__(512, 1)
       QIter it;
       q_iter_init(it, p.rd, k0, meta_b, use_seg);
       int n = 0;
-      for (int32_t q = q_iter_next(it, p.rd); q >= 0; q = q_iter_next(it, p.rd), ++n) {
+      for (int32_t q = q_iter_next_warp(it, p.rd); q >= 0; q = q_iter_next_warp(it, p.rd), ++n) {
         const int s = n & 1;
         if (!ra_wait_warp(bar(L::B_DQFULL + s), (n >> 1) & 1, abort_flag)) break;
         tc_fence_after();

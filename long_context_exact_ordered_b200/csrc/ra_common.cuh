@@ -96,29 +96,66 @@ RA_HD void kv_iter_init(KvIter& it, const RingDesc& rd, int64_t q_first, int64_t
   }
 }
 
+// Whether KV tile metadata m can hold a pair visible to the iterator's query rows.
+RA_HD bool kv_tile_visible(const KvIter& it, int4 m) {
+  if (it.use_seg && (m.y < it.q_seg_min || m.x > it.q_seg_max)) return false;
+  if (it.use_bias && !(m.z & kMetaAnyFinite)) return false;
+  return true;
+}
+
+// Move to the next ring step's tile range; false once the ring is closed.
+RA_HD bool kv_iter_step(KvIter& it, const RingDesc& rd) {
+  if (++it.step >= rd.P) return false;
+  int32_t src = it.r - rd.order[it.step];
+  src %= rd.P;
+  if (src < 0) src += rd.P;
+  int64_t a = (int64_t)src * rd.blk, b = (int64_t)(src + 1) * rd.blk;
+  it.tile = (int32_t)ceil_div64(a, kTile);
+  int64_t e = ceil_div64(b, kTile);
+  if (e > it.t_cap + 1) e = it.t_cap + 1;
+  it.tile_end = (int32_t)e;
+  return true;
+}
+
 // Next KV tile index in ring order, or -1 when the ring is closed.
 RA_HD int32_t kv_iter_next(KvIter& it, const RingDesc& rd) {
   while (true) {
     while (it.tile < it.tile_end) {
       int32_t t = it.tile++;
-      if (it.meta) {
-        int4 m = load_meta(it.meta + t);
-        if (it.use_seg && (m.y < it.q_seg_min || m.x > it.q_seg_max)) continue;
-        if (it.use_bias && !(m.z & kMetaAnyFinite)) continue;
-      }
+      if (it.meta && !kv_tile_visible(it, load_meta(it.meta + t))) continue;
       return t;
     }
-    if (++it.step >= rd.P) return -1;
-    int32_t src = it.r - rd.order[it.step];
-    src %= rd.P;
-    if (src < 0) src += rd.P;
-    int64_t a = (int64_t)src * rd.blk, b = (int64_t)(src + 1) * rd.blk;
-    it.tile = (int32_t)ceil_div64(a, kTile);
-    int64_t e = ceil_div64(b, kTile);
-    if (e > it.t_cap + 1) e = it.t_cap + 1;
-    it.tile_end = (int32_t)e;
+    if (!kv_iter_step(it, rd)) return -1;
   }
 }
+
+#ifdef __CUDACC__
+// kv_iter_next for a converged warp whose lanes all hold the same iterator:
+// the lanes test 32 candidate tiles at once, so a run of skipped tiles costs
+// one metadata round trip per 32 tiles instead of one per tile.  Returns the
+// same sequence as kv_iter_next.
+__device__ __forceinline__ int32_t kv_iter_next_warp(KvIter& it, const RingDesc& rd) {
+  const int lane = threadIdx.x & 31;
+  while (true) {
+    if (!it.meta) {
+      if (it.tile < it.tile_end) return it.tile++;
+    } else {
+      while (it.tile < it.tile_end) {
+        const int32_t t = it.tile + lane;
+        const bool vis = t < it.tile_end && kv_tile_visible(it, load_meta(it.meta + t));
+        const unsigned hit = __ballot_sync(0xffffffffu, vis);
+        if (hit) {
+          const int32_t first = it.tile + __ffs(hit) - 1;
+          it.tile = first + 1;
+          return first;
+        }
+        it.tile += 32;
+      }
+    }
+    if (!kv_iter_step(it, rd)) return -1;
+  }
+}
+#endif
 
 // Backward direction of the same ring: a key/value tile of ring block src
 // meets the query blocks (src + order[t]) mod P at steps t = 0, 1, ...
@@ -156,26 +193,58 @@ RA_HD void q_iter_init(QIter& it, const RingDesc& rd, int64_t k_first, const int
   }
 }
 
+RA_HD bool q_tile_visible(const QIter& it, int32_t q) {
+  const int4 m = load_meta(it.meta + (int64_t)q * kQTileBwd / kTile);
+  return !(m.y < it.k_seg_min || m.x > it.k_seg_max);
+}
+
+RA_HD bool q_iter_step(QIter& it, const RingDesc& rd) {
+  if (++it.step >= rd.P) return false;
+  int32_t r = (it.src + rd.order[it.step]) % rd.P;
+  int64_t a = (int64_t)r * rd.blk, b = (int64_t)(r + 1) * rd.blk;
+  int64_t lo = ceil_div64(a, kQTileBwd), hi = ceil_div64(b, kQTileBwd);
+  if (hi > it.nqt) hi = it.nqt;
+  if (lo < it.q_min) lo = it.q_min;
+  it.tile = (int32_t)lo;
+  it.tile_end = (int32_t)(hi > lo ? hi : lo);
+  return true;
+}
+
 RA_HD int32_t q_iter_next(QIter& it, const RingDesc& rd) {
   while (true) {
     while (it.tile < it.tile_end) {
       int32_t q = it.tile++;
-      if (it.meta) {
-        int4 m = load_meta(it.meta + (int64_t)q * kQTileBwd / kTile);
-        if (m.y < it.k_seg_min || m.x > it.k_seg_max) continue;
-      }
+      if (it.meta && !q_tile_visible(it, q)) continue;
       return q;
     }
-    if (++it.step >= rd.P) return -1;
-    int32_t r = (it.src + rd.order[it.step]) % rd.P;
-    int64_t a = (int64_t)r * rd.blk, b = (int64_t)(r + 1) * rd.blk;
-    int64_t lo = ceil_div64(a, kQTileBwd), hi = ceil_div64(b, kQTileBwd);
-    if (hi > it.nqt) hi = it.nqt;
-    if (lo < it.q_min) lo = it.q_min;
-    it.tile = (int32_t)lo;
-    it.tile_end = (int32_t)(hi > lo ? hi : lo);
+    if (!q_iter_step(it, rd)) return -1;
   }
 }
+
+#ifdef __CUDACC__
+// q_iter_next for a converged warp (same contract as kv_iter_next_warp).
+__device__ __forceinline__ int32_t q_iter_next_warp(QIter& it, const RingDesc& rd) {
+  const int lane = threadIdx.x & 31;
+  while (true) {
+    if (!it.meta) {
+      if (it.tile < it.tile_end) return it.tile++;
+    } else {
+      while (it.tile < it.tile_end) {
+        const int32_t q = it.tile + lane;
+        const bool vis = q < it.tile_end && q_tile_visible(it, q);
+        const unsigned hit = __ballot_sync(0xffffffffu, vis);
+        if (hit) {
+          const int32_t first = it.tile + __ffs(hit) - 1;
+          it.tile = first + 1;
+          return first;
+        }
+        it.tile += 32;
+      }
+    }
+    if (!q_iter_step(it, rd)) return -1;
+  }
+}
+#endif
 
 // Whether a (query tile, KV tile) pair needs the per-element mask: a causal
 // diagonal, a partly-out-of-range KV tile, or mixed segment ids.

@@ -149,32 +149,43 @@ __global__ void __launch_bounds__(384, 1)
   regs_dec<L::REGS_LOW>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      mbar_arrive_expect_tx(bar(L::B_Q), 2 * L::TILE_BYTES);
-      for (int qt = 0; qt < 2; ++qt)
-        for (int c = 0; c < L::KCH; ++c)
-          tma_load_4d(sbase + L::OFF_Q + qt * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_q, bar(L::B_Q), c * 64, h,
-                      (int)(q0 + qt * kTile), b);
+    // The whole warp runs the loop (its lanes scan 32 KV tiles per metadata
+    // round trip, kv_iter_next_warp); one elected lane issues the copies.
+    {
+      if (elect_one()) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        mbar_arrive_expect_tx(bar(L::B_Q), 2 * L::TILE_BYTES);
+        for (int qt = 0; qt < 2; ++qt)
+          for (int c = 0; c < L::KCH; ++c)
+            tma_load_4d(sbase + L::OFF_Q + qt * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_q, bar(L::B_Q), c * 64, h,
+                        (int)(q0 + qt * kTile), b);
+      }
+      __syncwarp();
       KvIter it;
       kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
       const uint64_t pol = l2_policy_evict_last();   // K/V tiles are re-read by every query pair of the head
       int nk = 0, nv = 0;   // K / V tiles issued
-      for (int32_t t = kv_iter_next(it, p.rd); t >= 0; t = kv_iter_next(it, p.rd)) {
+      for (int32_t t = kv_iter_next_warp(it, p.rd); t >= 0; t = kv_iter_next_warp(it, p.rd)) {
         const int ks = nk % L::KS, vs = nv % L::VS;
-        if (nk >= L::KS && !ra_wait(bar(L::B_KEMPTY + ks), ((nk / L::KS) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::B_KFULL + ks), L::TILE_BYTES);
-        for (int c = 0; c < L::KCH; ++c)
-          tma_load_4d_hint(sbase + L::OFF_K + ks * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_k, bar(L::B_KFULL + ks),
-                           c * 64, h, t * kTile, b, pol);
+        if (nk >= L::KS && !ra_wait_warp(bar(L::B_KEMPTY + ks), ((nk / L::KS) & 1) ^ 1, abort_flag)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(L::B_KFULL + ks), L::TILE_BYTES);
+          for (int c = 0; c < L::KCH; ++c)
+            tma_load_4d_hint(sbase + L::OFF_K + ks * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_k, bar(L::B_KFULL + ks),
+                             c * 64, h, t * kTile, b, pol);
+        }
+        __syncwarp();
         ++nk;
-        if (nv >= L::VS && !ra_wait(bar(L::B_VEMPTY + vs), ((nv / L::VS) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(L::B_VFULL + vs), L::TILE_BYTES);
-        for (int c = 0; c < L::KCH; ++c)
-          tma_load_4d_hint(sbase + L::OFF_V + vs * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_v, bar(L::B_VFULL + vs),
-                           c * 64, h, t * kTile, b, pol);
+        if (nv >= L::VS && !ra_wait_warp(bar(L::B_VEMPTY + vs), ((nv / L::VS) & 1) ^ 1, abort_flag)) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar(L::B_VFULL + vs), L::TILE_BYTES);
+          for (int c = 0; c < L::KCH; ++c)
+            tma_load_4d_hint(sbase + L::OFF_V + vs * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_v, bar(L::B_VFULL + vs),
+                             c * 64, h, t * kTile, b, pol);
+        }
+        __syncwarp();
         ++nv;
       }
       // Drain: every load issued must land before the block may exit.
@@ -210,7 +221,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       KvIter it;
       kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
-      int32_t t = kv_iter_next(it, p.rd);
+      int32_t t = kv_iter_next_warp(it, p.rd);
       bool ok = ra_wait_warp(bar(L::B_Q), 0, abort_flag);
       if (ok && t >= 0) {
         ok = ra_wait_warp(bar(L::B_KFULL + 0), 0, abort_flag);
@@ -223,7 +234,7 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit_w(bar(L::B_KEMPTY + 0));
         }
         for (int n = 0; ok; ++n) {
-          const int32_t tn = kv_iter_next(it, p.rd);
+          const int32_t tn = kv_iter_next_warp(it, p.rd);
           const bool last = tn < 0;
           const int vs = n % L::VS, ks1 = (n + 1) % L::KS;
           const uint32_t ph = n & 1;
@@ -293,7 +304,7 @@ __global__ void __launch_bounds__(384, 1)
 #endif
     int n = 0;
     bool ok = true;
-    for (int32_t t = kv_iter_next(it, p.rd); t >= 0; t = kv_iter_next(it, p.rd), ++n) {
+    for (int32_t t = kv_iter_next_warp(it, p.rd); t >= 0; t = kv_iter_next_warp(it, p.rd), ++n) {
       if (!(ok = ra_wait_warp(bar(L::B_SFULL + qt), n & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t sr[128];
