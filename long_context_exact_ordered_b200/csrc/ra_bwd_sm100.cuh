@@ -367,6 +367,8 @@ __global__ void __launch_bounds__(512, 1)
         const int st = n % L::NS, s = n & 1;
         const uint32_t slot = trow + s * L::SLOT_COLS;
         const int64_t q0 = (int64_t)q * L::QT;
+        // the query tile's metadata load is issued before the waits, so it lands meanwhile
+        const int4 qm = meta_b ? load_meta(meta_b + q0 / kTile) : make_int4(0, 0, 3, 0);
         if (!(ok = ra_wait_warp(bar(L::B_QF + st), (n / L::NS) & 1, abort_flag))) break;
         if (!(ok = ra_wait_warp(bar(L::B_SFULL + s), (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
@@ -386,7 +388,6 @@ __global__ void __launch_bounds__(512, 1)
           ffma2(x[c], x[c + 1], x[c], x[c + 1], sc, sc, b0, b1);
         }
         // per-element mask on causal-diagonal / ragged / mixed-segment tiles
-        const int4 qm = meta_b ? load_meta(meta_b + q0 / kTile) : make_int4(0, 0, 3, 0);
         const bool need_causal = cbs > 0 && q0 < k_last_blk;
         const bool need_ragged = (q0 + L::QT > S) || (k0 + kTile > S);
         const bool need_seg = use_seg && !(qm.x == qm.y && km.x == km.y && qm.x == km.x);

@@ -305,6 +305,8 @@ __global__ void __launch_bounds__(384, 1)
     int n = 0;
     bool ok = true;
     for (int32_t t = kv_iter_next_warp(it, p.rd); t >= 0; t = kv_iter_next_warp(it, p.rd), ++n) {
+      // the tile's metadata load is issued before the wait, so it lands while S is computed
+      const int4 km = meta_b ? load_meta(meta_b + t) : make_int4(0, 0, 3, 0);
       if (!(ok = ra_wait_warp(bar(L::B_SFULL + qt), n & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t sr[128];
@@ -318,7 +320,6 @@ __global__ void __launch_bounds__(384, 1)
       float* x = reinterpret_cast<float*>(sr);
 
       const int64_t k0 = (int64_t)t * kTile;
-      const int4 km = meta_b ? load_meta(meta_b + t) : make_int4(0, 0, 3, 0);
       // Scores stay raw (the scale is folded into the exponent's FMA) unless a
       // non-zero bias must be added first; loads are issued 32 keys at a time
       // (the empty asm keeps the compiler from hoisting all 128 and spilling).
