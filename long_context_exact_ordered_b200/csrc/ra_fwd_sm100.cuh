@@ -60,8 +60,8 @@ struct FwdLayout {
   static constexpr int B_VFULL = B_KEMPTY + KS;
   static constexpr int B_VEMPTY = B_VFULL + VS;
   static constexpr int B_SFULL = B_VEMPTY + VS;      // [2]
-  static constexpr int B_PFULL = B_SFULL + 2;        // [2]
-  static constexpr int B_PVDONE = B_PFULL + 2;       // [2]
+  static constexpr int B_PFULL = B_SFULL + 2;        // [2][2]: P of keys 0-63 / 64-127 written, per query tile
+  static constexpr int B_PVDONE = B_PFULL + 4;       // [2]
   static constexpr int B_DRAIN = B_PVDONE + 2;       // issuer's final commit
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;   // tmem slot, abort flag
@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < L::VS; ++i) { mbar_init(bar(L::B_VFULL + i), 1); mbar_init(bar(L::B_VEMPTY + i), 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(L::B_SFULL + i), 1);
-      mbar_init(bar(L::B_PFULL + i), 128);
+      mbar_init(bar(L::B_PFULL + 2 * i), 4);       // one arrive per softmax warp
+      mbar_init(bar(L::B_PFULL + 2 * i + 1), 4);
       mbar_init(bar(L::B_PVDONE + i), 1);
     }
     mbar_init(bar(L::B_DRAIN), 1);
@@ -212,12 +213,14 @@ __global__ void __launch_bounds__(384, 1)
                  kk > 0);
         }
       };
-      auto issue_pv = [&](int qt, int vs, bool acc) {
+      auto issue_pv = [&](int qt, int vs, int key_half, bool acc) {   // keys 64*key_half .. +63
         const uint32_t va = sbase + L::OFF_V + vs * L::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
+        for (int k = 0; k < kTile / 32; ++k) {
+          const int kk = key_half * (kTile / 32) + k;
           mma_ts_w(tO[qt], tS[qt] + kk * 8, smem_desc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), IDESC_PV,
-                 (acc || kk > 0) ? 1u : 0u);
+                   (acc || k > 0) ? 1u : 0u);
+        }
       };
       KvIter it;
       kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
@@ -240,9 +243,14 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t ph = n & 1;
           if (!(ok = ra_wait_warp(bar(L::B_VFULL + vs), (n / L::VS) & 1, abort_flag))) break;
           // query tile 0
+          // PV in two halves of the keys: the first runs while the softmax
+          // still computes P for the second
           if (!(ok = ra_wait_warp(bar(L::B_PFULL + 0), ph, abort_flag))) break;
           tc_fence_after();
-          issue_pv(0, vs, n > 0);
+          issue_pv(0, vs, 0, n > 0);
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 1), ph, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(0, vs, 1, true);
           mma_commit_w(bar(L::B_PVDONE + 0));
           if (!last) {
             // S0(n+1) overwrites the TMEM columns PV0(n) reads P0 from; the
@@ -253,9 +261,12 @@ __global__ void __launch_bounds__(384, 1)
             mma_commit_w(bar(L::B_SFULL + 0));
           }
           // query tile 1
-          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 1), ph, abort_flag))) break;
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 2), ph, abort_flag))) break;
           tc_fence_after();
-          issue_pv(1, vs, n > 0);
+          issue_pv(1, vs, 0, n > 0);
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 3), ph, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(1, vs, 1, true);
           mma_commit_w(bar(L::B_PVDONE + 1));
           mma_commit_w(bar(L::B_VEMPTY + vs));
           if (!last) {
@@ -421,11 +432,13 @@ __global__ void __launch_bounds__(384, 1)
           pk[(c >> 1) + 1] = pack_bf16x2(e2, e3);
         }
         tmem_st32(tS_row + half * 32, pk);
+        // P of this half of the keys is in TMEM: the MMA warp may start its half of PV
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_PFULL + 2 * qt + half));
       }
       l += (l0 + l1) + (l2 + l3);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_PFULL + qt));
     }
     // ---------------------------------------------------------- epilogue
     if (ok && n > 0) ok = ra_wait_warp(bar(L::B_PVDONE + qt), (n - 1) & 1, abort_flag);
