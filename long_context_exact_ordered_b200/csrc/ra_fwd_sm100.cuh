@@ -9,8 +9,10 @@
 // one), loaded by TMA.
 //
 // Roles (384 threads):
-//   warp 0      TMA producer (one lane): Q pair once, then K_t, V_t per tile.
-//   warp 1      TMEM owner; one lane issues every tcgen05.mma:
+//   warp 0      TMA producer (the whole warp walks the schedule, one elected
+//               lane issues copies): Q pair once, then K_t, V_t per tile.
+//   warp 1      TMEM owner; the whole warp runs the issue loop and one
+//               elected lane issues every tcgen05.mma:
 //                 S_q = Q_q K_t^T  (SS form, both K-major, M=N=128, fp32 in TMEM)
 //                 O_q += P_q V_t   (TS form: P from TMEM, V MN-major from SMEM)
 //   warps 4-7   softmax for query tile 0, warps 8-11 for query tile 1: thread
@@ -30,7 +32,9 @@
 // softmax 1 works on S1(t) the tensor core runs PV0/S0, and vice versa.
 // S_q(t+1) reuses the TMEM columns holding P_q(t); it is issued by the same
 // thread right behind PV_q(t) and the tensor pipe executes a thread's MMAs
-// in issue order.
+// in issue order.  P_q(t) is signalled per half of the keys and PV_q(t) is
+// issued in two halves, so the first half runs while the softmax still
+// computes P for the second.
 #pragma once
 
 #include <cuda.h>
