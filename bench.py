@@ -136,6 +136,28 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows), "power_w_max": max(power) if power else None}
 
 
+def mufu_rate(dev):
+    """ex2 per clock per SM from the debug build's microbenchmark (None if that build is absent)."""
+    import torch
+
+    try:
+        from long_context_exact_ordered_b200 import _lib
+
+        dbg = _lib.load_count()
+    except (ImportError, OSError, AttributeError):
+        return None
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    cycles = torch.zeros(sms, dtype=torch.int64, device=dev)
+    sink = torch.zeros(512, dtype=torch.float32, device=dev)
+    iters = 4096
+    s = torch.cuda.current_stream(dev).cuda_stream
+    for _ in range(2):
+        if dbg.ra_debug_ex2_rate(iters, sms, cycles.data_ptr(), sink.data_ptr(), s) != 0:
+            return None
+    torch.cuda.synchronize(dev)
+    return 512 * 8 * iters / cycles.double().mean().item(), sms
+
+
 def kernel_sources_sha256() -> str:
     h = hashlib.sha256()
     for f in KERNEL_SRCS:
@@ -245,6 +267,14 @@ def run_ours(args):
 
     peaks, peak_src = load_peaks()
     traffic, traffic_note = traffic_per_launch()
+    # the forward's co-ceiling: one MUFU ex2 per visible pair, measured live
+    mr = mufu_rate(dev)
+    mufu = None
+    if mr is not None:
+        rate, sms = mr
+        mhz = (clocks or {}).get("sm_mhz") or 0
+        mufu = {"ex2_per_clk_per_sm": round(rate, 2), "microbenchmark": "ra_debug_ex2_rate (libringattn_count.so)",
+                "fwd_cap_tflops_at_sm_mhz": round(rate * sms * mhz * 1e6 * 4 * w.D / 1e12, 1) if mhz else None}
     fwd_tf = fl_f / (t_f / 1e3) / 1e12
     achieved = fwd_tf if fwd_only else fl_b / (t_b / 1e3) / 1e12
     if fwd_only:
@@ -270,6 +300,7 @@ def run_ours(args):
         "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": None if fwd_only else round(achieved, 2),
         "frac_of_burst_peak_fwd_bwd": round(value / world / burst, 4),
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "roofline": roofline,
+        "mufu": mufu,
         "visible_pairs": n_vis,
     }
     if not args.no_cpu_baseline and rank == 0 and world == 1:

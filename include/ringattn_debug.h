@@ -11,6 +11,7 @@
  * for every row they own, the pairs their own tile skipping and per-element
  * masking let into the softmax (a score that is still finite there), so a
  * test can compare those counts bit for bit with an integer reference.
+ * It also carries a MUFU exp2 throughput microbenchmark.
  */
 #ifndef RINGATTN_DEBUG_H
 #define RINGATTN_DEBUG_H
@@ -37,6 +38,15 @@ extern "C" {
  * A process-wide setting: not for concurrent use from several threads.
  * Always returns RA_OK. */
 int ra_debug_set_counts(int32_t* fwd_row_counts, int32_t* bwd_col_counts);
+
+/* MUFU exp2 throughput microbenchmark (the forward's co-bound: one ex2 per
+ * visible pair).  Launches `blocks` CTAs of 512 threads (one per SM when
+ * blocks equals the SM count); each thread runs `iters` rounds of 8
+ * independent ex2.approx operations, and CTA i writes its elapsed SM clock
+ * cycles to cycles[i] (DEVICE, `blocks` entries).  sink: DEVICE float[512],
+ * never read (keeps the work live).  ex2 per clock per SM =
+ * 512 * 8 * iters / cycles[i].  RA_ERR_NULL / RA_ERR_SHAPE on bad arguments. */
+int ra_debug_ex2_rate(int32_t iters, int32_t blocks, long long* cycles, float* sink, void* stream);
 
 #ifdef __cplusplus
 }

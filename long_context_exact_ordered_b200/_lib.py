@@ -112,6 +112,9 @@ def load_count() -> ctypes.CDLL:
             fn.argtypes = args
         lib.ra_debug_set_counts.restype = ctypes.c_int
         lib.ra_debug_set_counts.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+        lib.ra_debug_ex2_rate.restype = ctypes.c_int
+        lib.ra_debug_ex2_rate.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p]
         _count_lib = lib
     return _count_lib
 

@@ -885,6 +885,36 @@ int ra_selftest_timeout(int64_t budget_cycles, void* stream) {
 }
 
 #ifdef RA_DEBUG_COUNT
+namespace {
+// MUFU ex2 throughput: 8 independent ex2 chains per thread (an FADD keeps
+// each chain bounded near -1); one CTA per SM records its cycle count.
+__global__ void __launch_bounds__(512, 1) debug_ex2_rate_kernel(int iters, long long* cycles, float* sink) {
+  float x[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) x[j] = -0.125f * (float)(j + 1) - 1e-3f * (float)threadIdx.x;
+  __syncthreads();
+  const long long t0 = clock64();
+  for (int i = 0; i < iters; ++i) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) x[j] = ex2_approx(x[j]) - 1.5f;
+  }
+  __syncthreads();
+  const long long t1 = clock64();
+  float acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc += x[j];
+  if (acc == 12345.f) sink[threadIdx.x] = acc;   // keeps the chains live
+  if (threadIdx.x == 0) cycles[blockIdx.x] = t1 - t0;
+}
+}  // namespace
+
+int ra_debug_ex2_rate(int32_t iters, int32_t blocks, long long* cycles, float* sink, void* stream) {
+  if (!cycles || !sink) return RA_ERR_NULL;
+  if (iters < 1 || blocks < 1) return RA_ERR_SHAPE;
+  debug_ex2_rate_kernel<<<(unsigned)blocks, 512, 0, static_cast<cudaStream_t>(stream)>>>(iters, cycles, sink);
+  return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
+}
+
 int ra_debug_set_counts(int32_t* fwd_row_counts, int32_t* bwd_col_counts) {
   g_dbg_fwd_rows = fwd_row_counts;
   g_dbg_bwd_cols = bwd_col_counts;
