@@ -38,6 +38,7 @@ from .attention import (  # noqa: F401
     attention_forward,
     attention_rows,
     causal_ok,
+    head_backward_cols,
     visible_count_cols,
     visible_count_rows,
     visible_mask,

@@ -74,19 +74,20 @@ def causal_ok(i, j, causal_block_size):
     return (i // c) >= (j // c)
 
 
-def visible_mask(rows, S, causal_block_size=None, seg_b=None, bias_b=None):
-    """Boolean visibility [len(rows), S] for query rows ``rows`` of one batch.
+def visible_mask(rows, S, causal_block_size=None, seg_b=None, bias_b=None, keys=None):
+    """Boolean visibility [len(rows), len(keys)] for query rows ``rows`` of one
+    batch against key positions ``keys`` (default: all S keys).
 
     ``seg_b`` / ``bias_b`` are that batch's segment ids / bias ([S]) or None.
     """
     rows = np.asarray(rows, dtype=np.int64)
-    keys = np.arange(S, dtype=np.int64)
+    keys = np.arange(S, dtype=np.int64) if keys is None else np.asarray(keys, dtype=np.int64)
     vis = causal_ok(rows[:, None], keys[None, :], causal_block_size)
     if seg_b is not None:
         seg_b = np.asarray(seg_b)
-        vis = vis & (seg_b[rows][:, None] == seg_b[None, :])
+        vis = vis & (seg_b[rows][:, None] == seg_b[keys][None, :])
     if bias_b is not None:
-        vis = vis & (np.asarray(bias_b, dtype=np.float64)[None, :] > -np.inf)
+        vis = vis & (np.asarray(bias_b, dtype=np.float64)[keys][None, :] > -np.inf)
     return vis
 
 
@@ -197,6 +198,38 @@ def _head_backward(qh, kh, vh, doh, oh, lse_h, rows_all, causal_block_size, seg_
             dk += scale * (dS.T @ qh[a:e])
             dv += P.T @ doh[a:e]
     return dq, dk, dv
+
+
+def head_backward_cols(qh, kh, vh, doh, oh, lse_h, cols, causal_block_size=None, seg_b=None, bias_b=None):
+    """dK and dV of one (b, h) at the key positions ``cols`` only.
+
+    The same sums as the full backward (dK_j = scale * sum_i dS_ij q_i,
+    dV_j = sum_i P_ij dO_i over every query row i), restricted to the chosen
+    keys, so sampled keys of a long sequence can be checked without the
+    whole backward.  ``oh`` / ``lse_h``: the head's forward output (as stored)
+    and log-sum-exp for all S rows.
+    """
+    S, D = kh.shape
+    scale = 1.0 / math.sqrt(D)
+    cols = np.asarray(cols, dtype=np.int64)
+    kc, vc = kh[cols], vh[cols]
+    bc = None if bias_b is None else np.where(np.isfinite(bias_b[cols]), bias_b[cols], 0.0)
+    dk = np.zeros((len(cols), D), dtype=np.float64)
+    dv = np.zeros((len(cols), D), dtype=np.float64)
+    for a, e in _row_chunks(S, max(len(cols), 1)):
+        rows = np.arange(a, e)
+        vis = visible_mask(rows, S, causal_block_size, seg_b, bias_b, keys=cols)
+        s = scale * (qh[a:e] @ kc.T)
+        if bc is not None:
+            s = s + bc[None, :]
+        lse_r = lse_h[a:e]
+        has = np.isfinite(lse_r)
+        P = np.where(vis & has[:, None], np.exp(s - np.where(has, lse_r, 0.0)[:, None]), 0.0)
+        Dl = np.sum(doh[a:e] * oh[a:e], axis=1)
+        dS = P * (doh[a:e] @ vc.T - Dl[:, None])
+        dk += scale * (dS.T @ qh[a:e])
+        dv += P.T @ doh[a:e]
+    return dk, dv
 
 
 def attention_backward(q, k, v, do, attention_bias=None, segment_ids=None, causal_block_size=None,

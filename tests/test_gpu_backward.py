@@ -22,7 +22,7 @@ import torch
 import oracle
 import workloads as W
 from checker import compare
-from gpu_util import to64, to_np
+from gpu_util import gather_rows, oracle_rows, to64, to_np
 
 pytestmark = pytest.mark.gpu
 ra = pytest.importorskip("long_context_exact_ordered_b200")
@@ -204,3 +204,48 @@ def test_config_causal64k_fwd_bwd():
     tol = 1e-2 * np.sqrt(w.S)
     np.testing.assert_allclose(to64(dk).sum(axis=1), 0.0, atol=tol)
     np.testing.assert_allclose(to64(dv).sum(axis=1), to64(inp["do"]).sum(axis=1), atol=tol)
+
+
+@pytest.mark.slow
+def test_config_causal128k_fwd_bwd():
+    """The bench's workload at full size, in the bench's launch configuration
+    (128K causal, B=1, H=32, D=128, P=8, chunks 512): O and LSE on 4096 sampled
+    rows, dQ on the same rows, dK / dV on 512 sampled keys of one seeded head
+    (including every ring-block boundary), and the invariants on all heads."""
+    w = W.WORKLOADS["causal128k"]
+    inp = W.make_inputs(w, dev())
+    o, lse, (dq, dk, dv) = run_both(w, inp)
+    samples = W.sample_rows(w, None, n=4096)
+    sel = (torch.as_tensor(samples[:, 0]), torch.as_tensor(samples[:, 2]), torch.as_tensor(samples[:, 1]))
+    # forward rows (one head's K / V on the host at a time)
+    ro, rl = oracle_rows(inp, samples, 1)
+    go, gl = gather_rows(o, lse, samples)
+    res = compare(go, ro, "bf16")
+    assert res.ok, f"o rows: {res}"
+    assert np.abs(gl - rl).max() <= 1e-3
+    # dQ rows, Delta from the stored output
+    got = to64(dq[sel])
+    want = np.zeros_like(got)
+    for h in np.unique(samples[:, 1]):
+        idx = np.nonzero(samples[:, 1] == h)[0]
+        rows = samples[idx, 2]
+        sub = np.stack([np.zeros_like(rows), np.zeros_like(rows), rows], axis=1)
+        qh, kh, vh, doh = (to64(inp[n][0, :, int(h)].contiguous())[None, :, None, :] for n in ("q", "k", "v", "do"))
+        want[idx] = _rows_grad_stored(qh, kh, vh, doh, sub)
+    res = compare(got, want, "bf16")
+    assert res.ok, f"dq rows: {res}"
+    # dK / dV on sampled keys of one head (its full forward gives every row's lse and stored o)
+    rng = np.random.default_rng(w.seed + 9)
+    h = int(rng.integers(0, w.H))
+    blk = w.S // w.P
+    edges = np.concatenate([np.arange(w.P) * blk, np.arange(1, w.P + 1) * blk - 1])
+    cols = np.unique(np.concatenate([edges, rng.choice(w.S, size=512 - len(edges), replace=False)]))
+    qh, kh, vh, doh = (to64(inp[n][0, :, h].contiguous()) for n in ("q", "k", "v", "do"))
+    o_h, l_h = oracle.attention_forward(qh[None, :, None], kh[None, :, None], vh[None, :, None], None, None, 1)
+    rk, rv = oracle.head_backward_cols(qh, kh, vh, doh, stored(o_h, torch.bfloat16)[0, :, 0], l_h[0, 0], cols, 1)
+    assert compare(to64(dk[0, torch.as_tensor(cols), h]), rk, "bf16").ok
+    assert compare(to64(dv[0, torch.as_tensor(cols), h]), rv, "bf16").ok
+    tol = 1e-2 * np.sqrt(w.S)
+    sum64 = lambda t: t.double().sum(dim=1).cpu().numpy()    # sums over tokens, in float64 on the device
+    np.testing.assert_allclose(sum64(dk), 0.0, atol=tol)
+    np.testing.assert_allclose(sum64(dv), sum64(inp["do"]), atol=tol)

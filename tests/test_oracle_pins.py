@@ -320,6 +320,22 @@ def test_backward_matches_finite_differences():
         np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-8, err_msg=name)
 
 
+def test_backward_on_sampled_keys_equals_full_backward():
+    """head_backward_cols (dK, dV at chosen keys) against the full backward,
+    itself pinned by finite differences above."""
+    S, D = 70, 8
+    q, k, v, do, seg, bias = tiny_case(S, D, seg=True, bias=True, neg_inf_bias=True)
+    c = 3
+    o, lse = oracle.attention_forward(q, k, v, bias, seg, c)
+    _, dk, dv = oracle.attention_backward(q, k, v, do, bias, seg, c, o=o, lse=lse)
+    cols = np.array([0, 1, 5, 33, 34, 69])
+    f = lambda x: np.asarray(x, dtype=np.float64)[0, :, 0]
+    gk, gv = oracle.head_backward_cols(f(q), f(k), f(v), f(do), f(o), np.asarray(lse)[0, 0], cols, c,
+                                       np.asarray(seg)[0], np.asarray(bias, dtype=np.float64)[0])
+    np.testing.assert_allclose(gk, dk[0, cols, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(gv, dv[0, cols, 0], rtol=0, atol=1e-12)
+
+
 def test_backward_invariants():
     S, D = 40, 8
     q, k, v, do, seg, bias = tiny_case(S, D, B=2, H=2, seg=True)
