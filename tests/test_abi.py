@@ -251,3 +251,21 @@ def test_train_step_host_argument_errors():
     t = _host_step()
     assert call(t, hpg=3) == 5                                              # 3 does not divide H = 4
     assert call(t, hpg=0) == 5
+
+
+def test_plain_c_client(tmp_path):
+    """The headers compile as C99 and the host-only entry points work from a C program."""
+    import shutil
+    import subprocess
+
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.dirname(_lib.LIB_PATH)
+    exe = str(tmp_path / "abi_host_only")
+    src = os.path.join(ROOT, "tests", "c", "abi_host_only.c")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), src, "-o", exe,
+                        "-L", pkg, "-lringattn", "-Wl,-rpath," + pkg], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
