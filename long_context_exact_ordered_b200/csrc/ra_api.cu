@@ -821,9 +821,6 @@ int ra_train_step_host(const ra_host_step* t, const ra_tensor* attention_bias, c
                              &t->dev_q, &t->dev_k, &t->dev_v, &t->dev_do, &t->dev_o, &t->dev_dq, &t->dev_dk,
                              &t->dev_dv};
   for (const ra_tensor* x : bshd)
-    if (!x->data) return RA_ERR_NULL;
-  if (!t->lse.data || !t->dev_lse.data) return RA_ERR_NULL;
-  for (const ra_tensor* x : bshd)
     if (x->ndim != 4) return RA_ERR_SHAPE;
   for (const ra_tensor* x : bshd)
     if (!same_shape(x, &t->q)) return x->dtype != t->q.dtype ? RA_ERR_DTYPE : RA_ERR_SHAPE;
@@ -836,7 +833,10 @@ int ra_train_step_host(const ra_host_step* t, const ra_tensor* attention_bias, c
     if (!contiguous_bhs(x)) return RA_ERR_STRIDE;
   }
   if (heads_per_group < 1 || H % heads_per_group) return RA_ERR_DIVISIBILITY;
-  if (B * S * H == 0) return RA_OK;
+  if (B * S * H == 0) return RA_OK;   // nothing to move or compute
+  for (const ra_tensor* x : bshd)
+    if (!x->data) return RA_ERR_NULL;
+  if (!t->lse.data || !t->dev_lse.data) return RA_ERR_NULL;
   cudaStream_t sc = static_cast<cudaStream_t>(compute_stream), si = static_cast<cudaStream_t>(h2d_stream),
                so = static_cast<cudaStream_t>(d2h_stream);
   EventPool pool;

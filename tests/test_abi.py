@@ -236,6 +236,10 @@ def test_train_step_host_argument_errors():
     t = _host_step()
     t.dev_dk.data = 0
     assert call(t) == 1                                                     # a missing buffer
+    t = _host_step(S=0)
+    for name in ("q", "dev_q", "lse"):
+        getattr(t, name).data = 0
+    assert call(t) == 0                                                     # empty problem: nothing to do
     t = _host_step()
     t.dq = T([1, 256, 4, 64], _lib.RA_F32)
     assert call(t) == 2                                                     # gradients take q's dtype
