@@ -98,8 +98,9 @@ def test_bf16_backward_full_parity(case):
         assert res.ok, f"{name}: {res}"
 
 
-def test_fp32_gradients_of_bf16_inputs_raw_tolerance():
-    w, inp = make(128, 1024, 4, 1, "packed", None, 1, 2)
+@pytest.mark.parametrize("D", [128, 64])
+def test_fp32_gradients_of_bf16_inputs_raw_tolerance(D):
+    w, inp = make(D, 1024, 4, 1, "packed", None, 1, 2)
     o, lse, (dq, dk, dv) = run_both(w, inp, grad_dtype=torch.float32)
     assert dq.dtype == torch.float32
     rq, rk, rv = oracle_grads(inp, 1)
