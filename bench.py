@@ -14,6 +14,12 @@ work divided by the slowest rank's device time ("scaling": "weak").
 
 Prints ONE JSON line on rank 0.  TFLOP/s counts only algorithmic work:
 4*D per visible (query, key) pair for the forward, 10*D for the backward.
+Besides the device-timed value it carries: "e2e", the same step through the
+host-buffer API (HostStep -> ra_train_step_host, pinned H2D / D2H copies
+inside the timed region); "roofline" for the backward kernel (measured peaks,
+DRAM bytes per launch from the committed full-size ncu capture); "mufu", the
+measured MUFU ex2 rate (the forward's second ceiling); "clocks" sampled during
+the timed region; and "cpu_baseline", the float64 oracle on a bounded sample.
 """
 
 from __future__ import annotations
