@@ -292,6 +292,7 @@ def run_ours(args):
                 "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                 "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a multi-second loop)",
                 "frac_of_burst_peak": round(achieved / burst, 4), "traffic": traffic,
+                "dram_gbs": (round(traffic / (t_b / 1e3) / 1e9, 1) if traffic is not None and t_b else None),
                 "traffic_note": traffic_note or "dram bytes per launch from the committed ncu capture",
                 "algorithmic_flop_per_launch": fl_f if fwd_only else fl_b}
     out = {
