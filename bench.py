@@ -6,11 +6,19 @@ for the 128K-token causal workload (B=1, H=32, D=128, S=131072, P=8 virtual
 ring ranks, chunks of 512, causal_block_size=1, bf16 N(0,1) inputs).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+                    [--workload NAME] [--mode fwdbwd|fwd|step] [--ring]
+                    [--no-e2e] [--no-cpu-baseline]
 
-Multi-GPU (torchrun, one process per GPU): the path does not shard, so every
-rank runs an independent replica of the workload; the value is all ranks'
-work divided by the slowest rank's device time ("scaling": "weak").
+--mode fwd times the forward alone; --mode step times the forward as the
+pages' ring runs it on one GPU: P virtual ranks x P per-step calls (ra_step,
+the tensor-core kernel in ring-step mode, each merging into its rank's fp32
+running state in HBM) plus ra_finalize per rank.
+
+Multi-GPU (torchrun, one process per GPU): by default every rank runs an
+independent replica of the workload; the value is all ranks' work divided by
+the slowest rank's device time ("scaling": "weak").  With --ring the
+sequence is sharded over the ranks instead and key/value blocks travel round
+the ring over NCCL (forward; "scaling": "strong").
 
 Prints ONE JSON line on rank 0.  TFLOP/s counts only algorithmic work:
 4*D per visible (query, key) pair for the forward, 10*D for the backward.
@@ -190,6 +198,15 @@ def traffic_per_launch():
 
 # ---------------------------------------------------------------- the step
 
+def workload_config(w, world):
+    """The "config" of the JSON line, the same for both arms."""
+    q_gb = w.B * w.S * w.H * w.D * 2 / 1e9
+    return {"workload": w.name, "description": w.description, "B": w.B, "H": w.H, "D": w.D, "S": w.S,
+            "ring_size": w.P, "chunk": w.chunk, "causal_block_size": w.causal_block_size,
+            "segments": w.segments, "bias": w.bias, "parallelism": f"replicas x{world}",
+            "l2": "no flush: every input tensor (%.2f GB) is larger than the 126 MB L2" % q_gb}
+
+
 def run_ours(args):
     import numpy as np
     import torch
@@ -221,12 +238,45 @@ def run_ours(args):
     ev_f = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
     ev_b = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
 
-    fwd_only = args.mode == "fwd"
+    step_mode = args.mode == "step"
+    fwd_only = args.mode in ("fwd", "step")
     if fwd_only:
         fl_b = 0.0
         launches_per_step = 1 + (1 if (bias is not None or seg is not None) else 0)
+    if step_mode:
+        # The forward as the pages' ring runs it, one ra_step per (rank, step):
+        # virtual rank r keeps query block r and meets key/value block
+        # (r - t) mod P at step t, merging into its own fp32 running state;
+        # then ra_finalize per rank.  Every state lives in HBM, as it would on
+        # a real ring rank.
+        P, blk = w.P, w.S // w.P
+        states = [ra.init_state(w.B, blk, w.H, w.D, dev) for _ in range(P)]
+        blocks = [slice(r * blk, (r + 1) * blk) for r in range(P)]
+        bias_b = [None if bias is None else bias[:, sl].contiguous() for sl in blocks]
+        seg_b = [None if seg is None else seg[:, sl].contiguous() for sl in blocks]
+        launches_per_step = P * P + P
+
+    def ring_of_steps():
+        for r in range(P):
+            acc, m, l = states[r]
+            acc.zero_()
+            m.fill_(float("-inf"))
+            l.zero_()
+            for t in range(P):
+                src = (r - t) % P
+                ra.ring_step(q[:, blocks[r]], k[:, blocks[src]], v[:, blocks[src]], r * blk, src * blk, acc, m, l,
+                             bias_blk=bias_b[src], seg_q=seg_b[r], seg_k=seg_b[src],
+                             causal_block_size=w.causal_block_size)
+            ra.finalize(acc, m, l, q.dtype, out=o[:, blocks[r]], lse=lse[:, :, blocks[r]])
 
     def step(prof=False):
+        if step_mode:
+            if prof:
+                ev_f[0].record()
+            ring_of_steps()
+            if prof:
+                ev_f[1].record()
+            return
         ra.ringattention(q, k, v, bias, seg, out=o, lse=lse, workspace=ws_f, prof_events=ev_f if prof else None, **kw)
         if not fwd_only:
             ra.ringattention_backward(q, k, v, o, lse, do, bias, seg, workspace=ws_b, out=grads,
@@ -299,11 +349,9 @@ def run_ours(args):
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
-        "config": {"workload": w.name, "description": w.description, "B": w.B, "H": w.H, "D": w.D, "S": w.S,
-                   "ring_size": w.P, "chunk": w.chunk, "causal_block_size": w.causal_block_size,
-                   "segments": w.segments, "bias": w.bias, "parallelism": f"replicas x{world}",
-                   "l2": "no flush: every input tensor (%.2f GB) is larger than the 126 MB L2" % (q.numel() * 2 / 1e9)},
-        "mode": "forward only" if fwd_only else "forward + backward",
+        "config": workload_config(w, world),
+        "mode": ("forward as P*P ring steps (ra_step) + finalize" if step_mode else
+                 "forward only" if fwd_only else "forward + backward"),
         "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": None if fwd_only else round(achieved, 2),
         "frac_of_burst_peak_fwd_bwd": round(value / world / burst, 4),
         "clocks": clocks, "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "roofline": roofline,
@@ -312,6 +360,86 @@ def run_ours(args):
     }
     if not args.no_cpu_baseline and rank == 0 and world == 1:
         out["cpu_baseline"] = cpu_baseline(w, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def run_ring(args):
+    """--ring: the forward with the sequence sharded over the N ranks, key/value
+    blocks exchanged round the ring over NCCL (long_context_exact_ordered_b200.ring,
+    zig-zag layout), ra_step on each rank's tensor cores.  Total work is fixed
+    ("scaling": "strong"); the value is the whole sequence's algorithmic
+    forward FLOP over the slowest rank's device time."""
+    import torch
+
+    import long_context_exact_ordered_b200 as ra
+    from long_context_exact_ordered_b200 import ring
+    import workloads as W
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    w = W.WORKLOADS[args.workload]
+    full = W.make_inputs(w, dev, with_grad_output=False)
+    n_vis = ra.count_visible_pairs(w.B, w.S, w.H, w.causal_block_size,
+                                   None if full["seg"] is None else full["seg"].cpu(),
+                                   None if full["bias"] is None else full["bias"].cpu())
+    mine = {n: (None if full[n] is None else ring.shard(full[n], rank, world, "zigzag"))
+            for n in ("q", "k", "v", "bias", "seg")}
+    del full
+    torch.cuda.empty_cache()
+    comm = torch.cuda.Stream(dev)
+
+    def step():
+        return ring.ring_attention_forward(mine["q"], mine["k"], mine["v"], mine["bias"], mine["seg"],
+                                           causal_block_size=w.causal_block_size, layout="zigzag",
+                                           comm_stream=comm)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if ra.device_status() != 0:
+        raise RuntimeError("device status word reports an error after warm-up")
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if not str(props.uuid).startswith("GPU-") else str(props.uuid))
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    fl = 4.0 * w.D * n_vis
+    value = fl * args.steps / (ms / 1e3) / 1e12
+    peaks, peak_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    per_gpu = value / world
+    calls = 4 * world + 2                  # ra_step calls (two query x two key chunks per ring step) + finalize
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "S": w.S, "causal_block_size": w.causal_block_size,
+                   "segments": w.segments, "parallelism": f"ring x{world} (sequence sharded, zig-zag, NCCL P2P)",
+                   "l2": "no flush: every rank's K / V shard is larger than the 126 MB L2" if w.S // world * w.H * w.D * 2 > 126e6
+                   else "no flush (small shards)"},
+        "mode": "ring forward across ranks", "clocks": clocks, "e2e": None,
+        "gpu_launches": calls * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "ra_fwd_sm100_kernel (ring-step mode)", "achieved": round(per_gpu, 2),
+                     "peak": burst, "unit": "TFLOP/s", "frac": round(per_gpu / burst, 4),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": None},
+        "visible_pairs": n_vis,
+    }
     if rank == 0:
         print(json.dumps(out), flush=True)
     if world > 1:
@@ -343,7 +471,7 @@ def run_e2e(args, w, inp, kw, dev, n_vis, world):
 
     one()
     torch.cuda.synchronize()
-    n = max(1, min(args.steps, 3))
+    n = max(1, args.steps)
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -382,10 +510,14 @@ def oracle_sample(w, rows_per_head, heads, seed):
         _ORACLE_INPUTS[w.name] = W.make_inputs(w, "cpu", with_grad_output=True)
     inp = _ORACLE_INPUTS[w.name]
     pairs = 0
+    # the inputs of a head, upcast to float64 once and kept (like the GPU's
+    # inputs resident in HBM); the oracle's own work is all that is timed
+    for h in heads:
+        if (w.name, h) not in _ORACLE_INPUTS:
+            _ORACLE_INPUTS[(w.name, h)] = tuple(inp[n][0, :, h].float().double().numpy() for n in ("q", "k", "v", "do"))
     t0 = time.perf_counter()
     for h in heads:
-        f = lambda n: inp[n][0, :, h].float().double().numpy()
-        qh, kh, vh, doh = f("q"), f("k"), f("v"), f("do")
+        qh, kh, vh, doh = _ORACLE_INPUTS[(w.name, h)]
         rows = np.sort(rng.choice(w.S, size=rows_per_head, replace=False))
         seg_b = None if inp["seg"] is None else inp["seg"][0].numpy()
         sub = np.stack([np.zeros_like(rows), np.zeros_like(rows), rows], axis=1)
@@ -406,13 +538,19 @@ def blas_threads():
         return len(os.sched_getaffinity(0))
 
 
-def cpu_baseline(w, budget_s=20.0):
-    """The oracle as it stands on this host's cores, on a bounded sample of the workload."""
-    # two-point calibration: the head's float64 conversion is a fixed cost per sample
+def calibrate_rows(w, budget_s):
+    """Query rows of head 0 that the oracle processes in about ``budget_s`` seconds
+    (two-point fit: a fixed cost per call plus a cost per row)."""
+    oracle_sample(w, 8, [0], seed=0)            # loads and upcasts the head's inputs once
     t8, _ = oracle_sample(w, 8, [0], seed=1)
     t64, _ = oracle_sample(w, 64, [0], seed=1)
     per_row = max((t64 - t8) / 56, 1e-6)
-    rows = int(max(8, min(8192, (budget_s - t8) / per_row)))
+    return int(max(8, min(8192, (budget_s - t8) / per_row)))
+
+
+def cpu_baseline(w, budget_s=20.0):
+    """The oracle as it stands on this host's cores, on a bounded sample of the workload."""
+    rows = calibrate_rows(w, budget_s)
     secs, pairs = oracle_sample(w, rows, [0], seed=2)
     val = 14.0 * w.D * pairs / secs / 1e12
     return {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -427,7 +565,8 @@ def run_reference(args):
     import workloads as W
 
     w = W.WORKLOADS[args.workload]
-    rows = args.ref_rows
+    # rows per step: about --ref-step-seconds of oracle work each (unless --ref-rows is given)
+    rows = args.ref_rows if args.ref_rows else calibrate_rows(w, args.ref_step_seconds)
     for i in range(args.warmup):
         oracle_sample(w, rows, [0], seed=100 + i)
     secs, pairs = 0.0, 0
@@ -441,8 +580,7 @@ def run_reference(args):
     out = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) bf16)",
-           "config": {"workload": w.name, "B": w.B, "H": w.H, "D": w.D, "S": w.S, "ring_size": w.P,
-                      "chunk": w.chunk, "causal_block_size": w.causal_block_size},
+           "config": workload_config(w, world),
            "cpu_baseline": {"value": val, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
@@ -455,17 +593,26 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="causal128k")
-    ap.add_argument("--mode", choices=["fwdbwd", "fwd"], default="fwdbwd",
-                    help="fwdbwd: one step = forward + backward (default); fwd: forward only")
+    ap.add_argument("--mode", choices=["fwdbwd", "fwd", "step"], default="fwdbwd",
+                    help="fwdbwd: one step = forward + backward (default); fwd: forward only; step: the forward "
+                         "as P*P per-step calls (ra_step, tensor cores) plus ra_finalize per rank")
+    ap.add_argument("--ring", action="store_true",
+                    help="forward with the sequence sharded over the N ranks (ring of NCCL exchanges) instead of "
+                         "N independent replicas")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0, help="seconds of oracle work for cpu_baseline")
-    ap.add_argument("--ref-rows", type=int, default=24, help="query rows per reference-arm step")
+    ap.add_argument("--ref-rows", type=int, default=0,
+                    help="query rows per reference-arm step (0: calibrated to --ref-step-seconds)")
+    ap.add_argument("--ref-step-seconds", type=float, default=4.0,
+                    help="oracle seconds per reference-arm step when calibrating the sample")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args)
+    elif args.ring:
+        run_ring(args)
     else:
         run_ours(args)
 

@@ -21,8 +21,9 @@
  *  - Tensors are described by ra_tensor: a pointer plus dtype, rank, shape
  *    and strides in ELEMENTS.  Data pointers are DEVICE pointers unless a
  *    parameter says "host".  The caller owns every buffer; the library never
- *    allocates device memory and keeps no state besides one device-side
- *    status word per device.
+ *    allocates device memory.  Its device-side state is one status word per
+ *    device, one word written by ra_selftest_timeout, and the fixed scratch
+ *    array of ra_forward_static (see there for how calls share it).
  *  - q, k, v, o, dO, dq, dk, dv are [B, S, H, D] (batch, token, head, head
  *    dim); the head dim must be contiguous (stride 1) and D in {64, 128}.
  *    bf16 tensors additionally need 16-byte aligned base pointers and
@@ -37,10 +38,17 @@
  *    key j is visible to query i iff floor(i/c) >= floor(j/c); c = 0 means
  *    non-causal.  Softmax scale is 1/sqrt(D).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
- *    default stream).  A non-zero return means nothing was launched and
- *    the outputs are unspecified.  No exception or exit crosses the ABI.
+ *    default stream).  Arguments, tensor maps and kernel attributes are
+ *    checked and prepared before the first launch, so an error found there
+ *    returns with nothing queued; only RA_ERR_CUDA from a failed launch can
+ *    follow launches already queued.  After a non-zero return the outputs
+ *    are unspecified.  No exception or exit crosses the ABI.
  *  - Errors detected on the device (a bounded wait that ran out) are
  *    recorded in the device status word; ra_get_device_status() reads it.
+ *  - Every call that launches work makes the device that holds its tensors
+ *    current for the calling thread (cudaSetDevice), which also makes that
+ *    device's primary context current: the calls work from threads that have
+ *    made no CUDA call yet (for example an autograd worker thread).
  */
 #ifndef RINGATTN_H_
 #define RINGATTN_H_
@@ -143,12 +151,26 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
  * sequence) attends to one visiting key/value block k_blk, v_blk [B,Sk,H,D]
  * (tokens k_off ..), updating the caller-held running state in place:
  *   o_acc fp32 [B,Sq,H,D] (unnormalised output), m, l fp32 [B,H,Sq]
- *   (running max in natural-log units, running sum).
+ *   (reference max in natural-log units, running sum), with
+ *   o_acc = sum_j e^(s_j - m) v_j and l = sum_j e^(s_j - m) over the keys
+ *   seen so far.
  * Initialise m = -inf, l = 0, o_acc = 0 before the first step; any step
- * order gives the same finalized result.  bias_blk: NULL or fp32 [B,Sk] for
- * the visiting keys; seg_q / seg_k: both NULL or int32 [B,Sq] / [B,Sk].
- * Only p->causal_block_size is used from p.  q/k/v bf16 or fp32 (fp32
- * arithmetic, CUDA cores). */
+ * order gives the same finalized result (ra_finalize).  bias_blk: NULL or
+ * fp32 [B,Sk] for the visiting keys; seg_q / seg_k: both NULL or int32
+ * [B,Sq] / [B,Sk].  Only p->causal_block_size is used from p; masks compare
+ * global positions.  m and l must have identical strides.
+ *  - The key/value side (k_blk, v_blk, bias_blk, seg_k) may have batch 1
+ *    while q_blk has batch B: that one block is then shared by every query
+ *    batch row, e.g. a cached prefix common to B requests ("Ring
+ *    Attention技术解析" §7: requests with the same prefix share its cache). 
+ *  - bf16 q/k/v: tensor cores (the forward kernel in ring-step mode: TMA
+ *    K/V stages, tcgen05 S = Q K^T and O += P V, exp2 online softmax), the
+ *    block's partial merged into the state in the kernel's epilogue.  o_acc
+ *    needs a 16-byte aligned base and 16-byte multiple strides.  m may sit
+ *    up to 8 ln 2 below the true running max (the kernel moves its
+ *    reference max lazily); l and o_acc are scaled to match, so the state
+ *    finalizes to the same result.
+ *  - fp32 q/k/v: CUDA cores in fp32 with accurate expf; m is the true max. */
 int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_blk, int64_t q_off, int64_t k_off,
             const ra_tensor* bias_blk, const ra_tensor* seg_q, const ra_tensor* seg_k, const ra_params* p,
             ra_tensor* o_acc, ra_tensor* m, ra_tensor* l, void* stream);
@@ -178,8 +200,10 @@ int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* 
  * B * ceil(S / 128) <= 65536 (for example B = 8 at 1M tokens).  Larger
  * problems return RA_ERR_STATIC_LIMIT and launch nothing.
  *  - The array is held by every GPU that loads the library until the process
- *    exits.  The first call on a device (with that device current) looks up
- *    the array's device address once; make that first call before any stream
+ *    exits.  Each call looks up the array's device address in the current
+ *    context (cudaGetSymbolAddress), so the address stays right after a
+ *    context is destroyed and created again.  The first call on a device may
+ *    load the library's device code; make that first call before any stream
  *    capture.
  *  - Every call shares the array and it keeps the last call's contents.  All
  *    of it that a call reads is rewritten by that call first, so nothing has
@@ -243,6 +267,13 @@ int ra_selftest_timeout(int64_t budget_cycles, void* stream);
 
 /* Static description of an error code (never NULL). */
 const char* ra_strerror(int code);
+
+/* The CUDA call and error behind the most recent RA_ERR_CUDA returned to
+ * the calling thread, as text (for example "kernel launch: invalid argument
+ * (cudaErrorInvalidValue, 1)"); an empty string if there was none.  The
+ * pointer is to thread-local storage, valid until the thread's next call
+ * into the library. */
+const char* ra_last_error_message(void);
 
 /* Host-only introspection (no device work).
  * Exact number of visible (query, key) pairs summed over batch and heads,

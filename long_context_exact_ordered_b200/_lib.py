@@ -69,6 +69,7 @@ SIGNATURES = {
     "ra_get_device_status": (ctypes.c_int, [_vp]),
     "ra_selftest_timeout": (ctypes.c_int, [ctypes.c_int64, _vp]),
     "ra_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "ra_last_error_message": (ctypes.c_char_p, []),
     "ra_count_visible_pairs": (ctypes.c_int64, [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
                                                  ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_float)]),
     "ra_ring_schedule": (ctypes.c_int64, [ctypes.c_int64, _P, ctypes.c_int64, ctypes.c_int64,
@@ -131,6 +132,10 @@ class RingAttnError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
         msg = load().ra_strerror(code).decode()
+        if code == 8:                                  # RA_ERR_CUDA: which call failed, and how
+            detail = load().ra_last_error_message().decode()
+            if detail:
+                msg = f"{msg}: {detail}"
         super().__init__(f"{where}: {ERRORS.get(code, code)} ({msg})")
 
 

@@ -168,7 +168,11 @@ def ringattention_backward(q, k, v, o, lse, do, attention_bias=None, segment_ids
 
 def ring_step(q_blk, k_blk, v_blk, q_off, k_off, o_acc, m, l, bias_blk=None, seg_q=None, seg_k=None,
               causal_block_size=None):
-    """One ring step, updating the running (o_acc, m, l) in place (see ra_step)."""
+    """One ring step, updating the running (o_acc, m, l) in place (see ra_step).
+
+    bf16 blocks run on the tensor cores (the forward kernel in ring-step
+    mode); fp32 blocks on CUDA cores.  Positions are global: the query block
+    starts at token ``q_off``, the visiting key/value block at ``k_off``."""
     p = _params(max(1, q_blk.shape[1]), None, None, causal_block_size, 1, None)
     tq, tk, tv = _tensor(q_blk), _tensor(k_blk), _tensor(v_blk)
     ta, tm, tl = _tensor(o_acc), _tensor(m), _tensor(l)
@@ -187,11 +191,13 @@ def init_state(B, S, H, D, device):
     return acc, m, l
 
 
-def finalize(o_acc, m, l, out_dtype=torch.bfloat16):
-    """(o_acc, m, l) -> (o, lse)."""
+def finalize(o_acc, m, l, out_dtype=torch.bfloat16, out=None, lse=None):
+    """(o_acc, m, l) -> (o, lse).  ``out`` / ``lse``: optional preallocated
+    outputs (any strides the C ABI accepts, e.g. views into larger tensors)."""
     B, S, H, D = o_acc.shape
-    o = torch.empty((B, S, H, D), dtype=out_dtype, device=o_acc.device)
-    lse = torch.empty((B, H, S), dtype=torch.float32, device=o_acc.device)
+    o = torch.empty((B, S, H, D), dtype=out_dtype, device=o_acc.device) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=o_acc.device)
     ta, tm, tl, to, tlse = _tensor(o_acc), _tensor(m), _tensor(l), _tensor(o), _tensor(lse)
     code = load().ra_finalize(ctypes.byref(ta), ctypes.byref(tm), ctypes.byref(tl), ctypes.byref(to),
                               ctypes.byref(tlse), _stream())

@@ -7,8 +7,8 @@
 #include <nvtx3/nvToolsExt.h>   // header-only; a no-op unless a profiler injects itself
 
 #include <cmath>
+#include <cstdio>
 #include <cstring>
-#include <mutex>
 #include <unordered_map>
 #include <vector>
 
@@ -23,7 +23,7 @@ using namespace ra;
 // Fixed scratch for ra_forward_static (tile metadata), one copy per device.
 // Host code must not pass this symbol to a kernel directly: on the host it is
 // only a stand-in, so its device address is looked up with
-// cudaGetSymbolAddress (per device, with that device current).
+// cudaGetSymbolAddress in the current context, on every call.
 static __device__ __align__(256) unsigned char g_ra_static_scratch[RA_STATIC_SCRATCH_BYTES];
 // Written only by the failure-path self-test kernel (1 = its wait gave up).
 static __device__ int g_ra_selftest_result;
@@ -36,6 +36,25 @@ static int32_t* g_dbg_bwd_cols = nullptr;
 #endif
 
 namespace {
+
+// ---------------------------------------------------------------- CUDA failures
+
+// What stood behind the last RA_ERR_CUDA returned to this thread (read by
+// ra_last_error_message).
+thread_local char t_last_error[192] = "";
+
+int cuda_fail(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return RA_OK;
+  std::snprintf(t_last_error, sizeof(t_last_error), "%s: %s (%s, %d)", what, cudaGetErrorString(e),
+                cudaGetErrorName(e), (int)e);
+  return RA_ERR_CUDA;
+}
+
+int cu_fail(CUresult r, const char* what) {
+  if (r == CUDA_SUCCESS) return RA_OK;
+  std::snprintf(t_last_error, sizeof(t_last_error), "%s: CUresult %d", what, (int)r);
+  return RA_ERR_CUDA;
+}
 
 // ---------------------------------------------------------------- validation
 
@@ -155,10 +174,23 @@ WsLayout ws_layout(int which, int64_t B, int64_t S, int64_t H, int64_t D, bool n
 
 // ---------------------------------------------------------------- device facts
 
-int device_cc_major() {
-  int dev = 0, major = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return -1;
+// Makes the device that holds `data` current for this thread and its primary
+// context current (the tensor-map encoder is a driver call and needs one: a
+// thread that has made no runtime call yet, such as an autograd worker, may
+// have none), then returns that device's compute-capability major, or -1
+// (the cause recorded) on failure.
+int bind_device(const void* data) {
+  cudaPointerAttributes a;
+  if (cuda_fail(cudaPointerGetAttributes(&a, data), "cudaPointerGetAttributes") != RA_OK) return -1;
+  int dev = a.device;
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) {
+    if (cuda_fail(cudaGetDevice(&dev), "cudaGetDevice") != RA_OK) return -1;
+  }
+  if (cuda_fail(cudaSetDevice(dev), "cudaSetDevice") != RA_OK) return -1;
+  int major = 0;
+  if (cuda_fail(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev), "cudaDeviceGetAttribute") !=
+      RA_OK)
+    return -1;
   return major;
 }
 
@@ -183,7 +215,7 @@ EncodeTiledFn encode_fn() {
 // bf16 [B, S, H, D] -> 4-D map (D, H, S, B), box 64 x 1 x rows x 1, 128-byte swizzle.
 int make_tmap_bshd(CUtensorMap* m, const ra_tensor* t, int rows) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return RA_ERR_CUDA;
+  if (!enc) return cu_fail(CUDA_ERROR_NOT_FOUND, "cuTensorMapEncodeTiled entry point");
   cuuint64_t dims[4] = {(cuuint64_t)t->shape[3], (cuuint64_t)t->shape[2], (cuuint64_t)t->shape[1],
                         (cuuint64_t)t->shape[0]};
   cuuint64_t strides[3] = {(cuuint64_t)t->stride[2] * 2, (cuuint64_t)t->stride[1] * 2, (cuuint64_t)t->stride[0] * 2};
@@ -192,24 +224,10 @@ int make_tmap_bshd(CUtensorMap* m, const ra_tensor* t, int rows) {
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, t->data, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? RA_OK : RA_ERR_CUDA;
+  return cu_fail(r, "cuTensorMapEncodeTiled (bf16 [B,S,H,D])");
 }
 
-int last_cuda() { return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA; }
-
-// fp32 [BH][S][D] workspace -> 3-D map (D, S, BH), box D x rows x 1, no swizzle.
-int make_tmap_dqacc(CUtensorMap* m, float* base, int64_t BH, int64_t S, int64_t D, int rows) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return RA_ERR_CUDA;
-  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)S * D * 4};
-  cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)rows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? RA_OK : RA_ERR_CUDA;
-}
+int last_cuda(const char* what = "kernel launch") { return cuda_fail(cudaGetLastError(), what); }
 
 // NVTX range around one entry point's host work (its launches show under it
 // in an nsys / ncu timeline).
@@ -255,134 +273,212 @@ int launch_meta(const MaskArgs& mk, int64_t B, const RingDesc& rd, int4* meta, c
   return last_cuda();
 }
 
-template <int D>
-int launch_fwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const MaskArgs& mk,
-                     const RingDesc& rd, const int4* meta, ra_tensor* o, ra_tensor* lse, cudaStream_t st) {
+// Shared-memory size attribute of the forward kernel, and the check that its
+// register split (setmaxnreg) fits in the registers the block launches with.
+template <int D, bool STEP>
+int fwd_kernel_attrs() {
+  using L = FwdLayout<D>;
+  RA_TRY(cuda_fail(cudaFuncSetAttribute(ra_fwd_sm100_kernel<D, STEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        L::SMEM_ALLOC),
+                   "cudaFuncSetAttribute (forward kernel)"));
+  cudaFuncAttributes fa;
+  RA_TRY(cuda_fail(cudaFuncGetAttributes(&fa, ra_fwd_sm100_kernel<D, STEP>), "cudaFuncGetAttributes (forward kernel)"));
+  if (128 * L::REGS_LOW + 256 * L::REGS_HIGH > L::THREADS * fa.numRegs) return RA_ERR_UNSUPPORTED;
+  return RA_OK;
+}
+
+// A kernel launch whose set-up (tensor maps, kernel attributes, register
+// split check) is done by prepare(), before any launch of the entry point,
+// so that every set-up error is returned with nothing queued on the stream.
+template <int D, bool STEP = false>
+struct FwdSm100Launch {
   using L = FwdLayout<D>;
   CUtensorMap tq, tk, tv;
-  RA_TRY(make_tmap_bshd(&tq, q, kTile));
-  RA_TRY(make_tmap_bshd(&tk, k, kTile));
-  RA_TRY(make_tmap_bshd(&tv, v, kTile));
   FwdParams prm;
-  std::memset(&prm, 0, sizeof(prm));
-  prm.rd = rd;
-  prm.B = (int32_t)q->shape[0];
-  prm.H = (int32_t)q->shape[2];
-  prm.npairs = (rd.ntiles + 1) / 2;
-  prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  prm.o = static_cast<__nv_bfloat16*>(o->data);
-  prm.o_sb = o->stride[0];
-  prm.o_ss = o->stride[1];
-  prm.o_sh = o->stride[2];
-  prm.lse = static_cast<float*>(lse->data);
-  prm.lse_sb = lse->stride[0];
-  prm.lse_sh = lse->stride[1];
-  prm.lse_ss = lse->stride[2];
-  prm.seg = mk.seg;
-  prm.seg_sb = mk.seg_sb;
-  prm.seg_ss = mk.seg_ss;
-  prm.bias = mk.bias;
-  prm.bias_sb = mk.bias_sb;
-  prm.bias_ss = mk.bias_ss;
-  prm.meta = meta;
+  int64_t grid = 0;
+
+  int prepare(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const MaskArgs& mk, const RingDesc& rd,
+              const int4* meta, ra_tensor* o, ra_tensor* lse) {
+    RA_TRY(make_tmap_bshd(&tq, q, kTile));
+    RA_TRY(make_tmap_bshd(&tk, k, kTile));
+    RA_TRY(make_tmap_bshd(&tv, v, kTile));
+    std::memset(&prm, 0, sizeof(prm));
+    prm.rd = rd;
+    prm.B = (int32_t)q->shape[0];
+    prm.H = (int32_t)q->shape[2];
+    prm.npairs = (rd.ntiles + 1) / 2;
+    prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    prm.o = static_cast<__nv_bfloat16*>(o->data);
+    prm.o_sb = o->stride[0];
+    prm.o_ss = o->stride[1];
+    prm.o_sh = o->stride[2];
+    prm.lse = static_cast<float*>(lse->data);
+    prm.lse_sb = lse->stride[0];
+    prm.lse_sh = lse->stride[1];
+    prm.lse_ss = lse->stride[2];
+    prm.seg = mk.seg;
+    prm.seg_sb = mk.seg_sb;
+    prm.seg_ss = mk.seg_ss;
+    prm.bias = mk.bias;
+    prm.bias_sb = mk.bias_sb;
+    prm.bias_ss = mk.bias_ss;
+    prm.meta = meta;
 #ifdef RA_DEBUG_COUNT
-  prm.dbg_count = g_dbg_fwd_rows;
+    prm.dbg_count = g_dbg_fwd_rows;
 #endif
-  const int64_t grid = (int64_t)prm.npairs * prm.B * prm.H;
-  if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(ra_fwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
-      cudaSuccess)
-    return RA_ERR_CUDA;
-  {
-    // The register split must fit in what the block is launched with.
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, ra_fwd_sm100_kernel<D>) != cudaSuccess) return RA_ERR_CUDA;
-    if (128 * L::REGS_LOW + 256 * L::REGS_HIGH > L::THREADS * fa.numRegs) return RA_ERR_UNSUPPORTED;
+    grid = (int64_t)prm.npairs * prm.B * prm.H;
+    if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
+    return fwd_kernel_attrs<D, STEP>();
   }
-  ra_fwd_sm100_kernel<D><<<(unsigned)grid, 384, L::SMEM_ALLOC, st>>>(tq, tk, tv, prm);
-  return last_cuda();
-}
+  // Ring-step mode: q_blk [B,Sq,H,D] at global token q_off against one
+  // visiting block k_blk, v_blk [B,Sk,H,D] at k_off, merged into (acc, m, l).
+  int prepare_step(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, int64_t q_off, int64_t k_off,
+                   int32_t cbs, const ra_tensor* bias, const ra_tensor* seg_q, const ra_tensor* seg_k,
+                   ra_tensor* acc, ra_tensor* m, ra_tensor* l) {
+    RA_TRY(make_tmap_bshd(&tq, q, kTile));
+    RA_TRY(make_tmap_bshd(&tk, k, kTile));
+    RA_TRY(make_tmap_bshd(&tv, v, kTile));
+    std::memset(&prm, 0, sizeof(prm));
+    const int64_t Sq = q->shape[1];
+    prm.rd.S = Sq;
+    prm.rd.blk = Sq;
+    prm.rd.P = 1;
+    prm.rd.ntiles = (int32_t)ceil_div64(Sq, kTile);
+    prm.rd.cbs = cbs;
+    prm.B = (int32_t)q->shape[0];
+    prm.H = (int32_t)q->shape[2];
+    prm.npairs = (prm.rd.ntiles + 1) / 2;
+    prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+    if (seg_q) {
+      prm.seg = static_cast<const int32_t*>(seg_q->data);
+      prm.seg_sb = seg_q->stride[0];
+      prm.seg_ss = seg_q->stride[1];
+      prm.seg_k = static_cast<const int32_t*>(seg_k->data);
+      prm.segk_sb = seg_k->stride[0];
+      prm.segk_ss = seg_k->stride[1];
+    }
+    if (bias) {
+      prm.bias = static_cast<const float*>(bias->data);
+      prm.bias_sb = bias->stride[0];
+      prm.bias_ss = bias->stride[1];
+    }
+    prm.Sk = k->shape[1];
+    prm.q_off = q_off;
+    prm.k_off = k_off;
+    prm.acc = static_cast<float*>(acc->data);
+    prm.acc_sb = acc->stride[0];
+    prm.acc_ss = acc->stride[1];
+    prm.acc_sh = acc->stride[2];
+    prm.m_state = static_cast<float*>(m->data);
+    prm.l_state = static_cast<float*>(l->data);
+    prm.ml_sb = m->stride[0];
+    prm.ml_sh = m->stride[1];
+    prm.ml_ss = m->stride[2];
+    grid = (int64_t)prm.npairs * prm.B * prm.H;
+    if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
+    return fwd_kernel_attrs<D, STEP>();
+  }
+  int launch(cudaStream_t st) const {
+    ra_fwd_sm100_kernel<D, STEP><<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, prm);
+    return last_cuda();
+  }
+};
 
 View4 view4(const ra_tensor* t) { return View4{t->data, t->stride[0], t->stride[1], t->stride[2]}; }
 OutView4 oview4(ra_tensor* t) { return OutView4{t->data, t->stride[0], t->stride[1], t->stride[2]}; }
 
 template <int D, typename T>
-int launch_fwd_simt(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const MaskArgs& mk,
-                    const RingDesc& rd, const int4* meta, ra_tensor* o, ra_tensor* lse, cudaStream_t st) {
+struct FwdSimtLaunch {
   SimtFwdArgs a;
-  std::memset(&a, 0, sizeof(a));
-  a.rd = rd;
-  a.B = (int)q->shape[0];
-  a.H = (int)q->shape[2];
-  a.scale = (float)(1.0 / std::sqrt((double)D));
-  a.mk = mk;
-  a.meta = meta;
-  a.q = view4(q);
-  a.k = view4(k);
-  a.v = view4(v);
-  a.o = oview4(o);
-  a.lse = static_cast<float*>(lse->data);
-  a.lse_sb = lse->stride[0];
-  a.lse_sh = lse->stride[1];
-  a.lse_ss = lse->stride[2];
-  const int smem = SimtSmem<D>::BYTES;
-  if (cudaFuncSetAttribute(simt_fwd_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return RA_ERR_CUDA;
-  dim3 grid((unsigned)ceil_div64(rd.S, kSimtRows), (unsigned)(a.B * a.H));
-  simt_fwd_kernel<D, T><<<grid, kSimtRows, smem, st>>>(a);
-  return last_cuda();
-}
+  dim3 grid;
+  static constexpr int kSmem = SimtSmem<D>::BYTES;
+
+  int prepare(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const MaskArgs& mk, const RingDesc& rd,
+              const int4* meta, ra_tensor* o, ra_tensor* lse) {
+    std::memset(&a, 0, sizeof(a));
+    a.rd = rd;
+    a.B = (int)q->shape[0];
+    a.H = (int)q->shape[2];
+    a.scale = (float)(1.0 / std::sqrt((double)D));
+    a.mk = mk;
+    a.meta = meta;
+    a.q = view4(q);
+    a.k = view4(k);
+    a.v = view4(v);
+    a.o = oview4(o);
+    a.lse = static_cast<float*>(lse->data);
+    a.lse_sb = lse->stride[0];
+    a.lse_sh = lse->stride[1];
+    a.lse_ss = lse->stride[2];
+    grid = dim3((unsigned)ceil_div64(rd.S, kSimtRows), (unsigned)(a.B * a.H));
+    return cuda_fail(cudaFuncSetAttribute(simt_fwd_kernel<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem),
+                     "cudaFuncSetAttribute (fp32 forward kernel)");
+  }
+  int launch(cudaStream_t st) const {
+    simt_fwd_kernel<D, T><<<grid, kSimtRows, kSmem, st>>>(a);
+    return last_cuda();
+  }
+};
 
 template <int D>
-int launch_bwd_sm100(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* d_o,
-                     const MaskArgs& mk, const RingDesc& rd, const int4* meta, const WsLayout& w, char* ws,
-                     ra_tensor* dk, ra_tensor* dv, cudaStream_t st) {
+struct BwdSm100Launch {
   using L = BwdLayout<D>;
-  CUtensorMap tq, tk, tv, tdo, tdq;
-  RA_TRY(make_tmap_bshd(&tq, q, L::QT));
-  RA_TRY(make_tmap_bshd(&tk, k, kTile));
-  RA_TRY(make_tmap_bshd(&tv, v, kTile));
-  RA_TRY(make_tmap_bshd(&tdo, d_o, L::QT));
-  RA_TRY(make_tmap_dqacc(&tdq, reinterpret_cast<float*>(ws + w.dqacc), q->shape[0] * q->shape[2], q->shape[1],
-                         L::D, L::QT));
+  CUtensorMap tq, tk, tv, tdo;
   BwdParams prm;
-  std::memset(&prm, 0, sizeof(prm));
-  prm.rd = rd;
-  prm.B = (int32_t)q->shape[0];
-  prm.H = (int32_t)q->shape[2];
-  prm.scale = (float)(1.0 / std::sqrt((double)L::D));
-  prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)L::D));
-  prm.lse2 = reinterpret_cast<const float*>(ws + w.lse2);
-  prm.delta = reinterpret_cast<const float*>(ws + w.delta);
-  prm.s_pad = w.s_pad;
-  prm.dqacc = reinterpret_cast<float*>(ws + w.dqacc);
-  prm.dk = dk->data;
-  prm.dk_sb = dk->stride[0];
-  prm.dk_ss = dk->stride[1];
-  prm.dk_sh = dk->stride[2];
-  prm.dv = dv->data;
-  prm.dv_sb = dv->stride[0];
-  prm.dv_ss = dv->stride[1];
-  prm.dv_sh = dv->stride[2];
-  prm.grad_bf16 = dk->dtype == RA_BF16;
-  prm.seg = mk.seg;
-  prm.seg_sb = mk.seg_sb;
-  prm.seg_ss = mk.seg_ss;
-  prm.bias = mk.bias;
-  prm.bias_sb = mk.bias_sb;
-  prm.bias_ss = mk.bias_ss;
-  prm.meta = meta;
+  int64_t grid = 0;
+
+  int prepare(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* d_o, const MaskArgs& mk,
+              const RingDesc& rd, const int4* meta, const WsLayout& w, char* ws, ra_tensor* dk, ra_tensor* dv) {
+    RA_TRY(make_tmap_bshd(&tq, q, L::QT));
+    RA_TRY(make_tmap_bshd(&tk, k, kTile));
+    RA_TRY(make_tmap_bshd(&tv, v, kTile));
+    RA_TRY(make_tmap_bshd(&tdo, d_o, L::QT));
+    std::memset(&prm, 0, sizeof(prm));
+    prm.rd = rd;
+    prm.B = (int32_t)q->shape[0];
+    prm.H = (int32_t)q->shape[2];
+    prm.scale = (float)(1.0 / std::sqrt((double)L::D));
+    prm.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)L::D));
+    prm.lse2 = reinterpret_cast<const float*>(ws + w.lse2);
+    prm.delta = reinterpret_cast<const float*>(ws + w.delta);
+    prm.s_pad = w.s_pad;
+    prm.dqacc = reinterpret_cast<float*>(ws + w.dqacc);
+    prm.dk = dk->data;
+    prm.dk_sb = dk->stride[0];
+    prm.dk_ss = dk->stride[1];
+    prm.dk_sh = dk->stride[2];
+    prm.dv = dv->data;
+    prm.dv_sb = dv->stride[0];
+    prm.dv_ss = dv->stride[1];
+    prm.dv_sh = dv->stride[2];
+    prm.grad_bf16 = dk->dtype == RA_BF16;
+    prm.seg = mk.seg;
+    prm.seg_sb = mk.seg_sb;
+    prm.seg_ss = mk.seg_ss;
+    prm.bias = mk.bias;
+    prm.bias_sb = mk.bias_sb;
+    prm.bias_ss = mk.bias_ss;
+    prm.meta = meta;
 #ifdef RA_DEBUG_COUNT
-  prm.dbg_count = g_dbg_bwd_cols;
+    prm.dbg_count = g_dbg_bwd_cols;
 #endif
-  const int64_t grid = (int64_t)rd.ntiles * prm.B * prm.H;
-  if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
-  if (cudaFuncSetAttribute(ra_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC) !=
-      cudaSuccess)
-    return RA_ERR_CUDA;
-  ra_bwd_sm100_kernel<D><<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, tdq, prm);
-  return last_cuda();
-}
+    grid = (int64_t)rd.ntiles * prm.B * prm.H;
+    if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
+    RA_TRY(cuda_fail(
+        cudaFuncSetAttribute(ra_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC),
+        "cudaFuncSetAttribute (backward kernel)"));
+    // The register split must fit in what the block is launched with.
+    cudaFuncAttributes fa;
+    RA_TRY(cuda_fail(cudaFuncGetAttributes(&fa, ra_bwd_sm100_kernel<D>), "cudaFuncGetAttributes (backward kernel)"));
+    if (128 * (L::REGS_WG0 + 2 * L::REGS_SOFTMAX + L::REGS_READOUT) > L::THREADS * fa.numRegs)
+      return RA_ERR_UNSUPPORTED;
+    return RA_OK;
+  }
+  int launch(cudaStream_t st) const {
+    ra_bwd_sm100_kernel<D><<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, prm);
+    return last_cuda();
+  }
+};
 
 template <int D, typename T>
 int launch_bwd_simt(const SimtBwdArgs& a, int64_t S, cudaStream_t st) {
@@ -457,27 +553,39 @@ int ra_forward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const
   const WsLayout w = ws_layout(0, B, S, H, D, need_meta);
   if (w.total > 0 && (!workspace || workspace_bytes < w.total)) return RA_ERR_WORKSPACE;
   if (w.total > 0 && reinterpret_cast<uintptr_t>(workspace) % 256) return RA_ERR_WORKSPACE;
-  if (dt == RA_BF16) {
-    const int major = device_cc_major();
-    if (major < 0) return RA_ERR_CUDA;
-    if (major != 10) return RA_ERR_UNSUPPORTED;
+  {
+    const int major = bind_device(q->data);
+    if (major < 0) return RA_ERR_CUDA;   // cause recorded by bind_device
+    if (dt == RA_BF16 && major != 10) return RA_ERR_UNSUPPORTED;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const MaskArgs mk = mask_args(attention_bias, segment_ids);
   int4* meta = need_meta ? reinterpret_cast<int4*>(static_cast<char*>(workspace) + w.meta) : nullptr;
-  if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
   const ProfScope prof(p, st);
-  prof.begin();
-  int rc;
+  // Set-up first (tensor maps, attributes), then the launches: a set-up
+  // error returns with nothing queued.
+  auto run = [&](auto& lc) -> int {
+    RA_TRY(lc.prepare(q, k, v, mk, rd, meta, o, lse));
+    if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
+    prof.begin();
+    const int rc = lc.launch(st);
+    prof.end();
+    return rc;
+  };
   if (dt == RA_BF16) {
-    rc = D == 64 ? launch_fwd_sm100<64>(q, k, v, mk, rd, meta, o, lse, st)
-                 : launch_fwd_sm100<128>(q, k, v, mk, rd, meta, o, lse, st);
-  } else {
-    rc = D == 64 ? launch_fwd_simt<64, float>(q, k, v, mk, rd, meta, o, lse, st)
-                 : launch_fwd_simt<128, float>(q, k, v, mk, rd, meta, o, lse, st);
+    if (D == 64) {
+      FwdSm100Launch<64> lc;
+      return run(lc);
+    }
+    FwdSm100Launch<128> lc;
+    return run(lc);
   }
-  prof.end();
-  return rc;
+  if (D == 64) {
+    FwdSimtLaunch<64, float> lc;
+    return run(lc);
+  }
+  FwdSimtLaunch<128, float> lc;
+  return run(lc);
 }
 
 int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* o,
@@ -517,16 +625,24 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   const WsLayout w = ws_layout(1, B, S, H, D, need_meta);
   if (!workspace || workspace_bytes < w.total || reinterpret_cast<uintptr_t>(workspace) % 256)
     return RA_ERR_WORKSPACE;
-  if (dt == RA_BF16) {
-    const int major = device_cc_major();
-    if (major < 0) return RA_ERR_CUDA;
-    if (major != 10) return RA_ERR_UNSUPPORTED;
+  {
+    const int major = bind_device(q->data);
+    if (major < 0) return RA_ERR_CUDA;   // cause recorded by bind_device
+    if (dt == RA_BF16 && major != 10) return RA_ERR_UNSUPPORTED;
   }
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const MaskArgs mk = mask_args(attention_bias, segment_ids);
   char* ws = static_cast<char*>(workspace);
   int4* meta = need_meta ? reinterpret_cast<int4*>(ws + w.meta) : nullptr;
   const bool tc_path = dt == RA_BF16;   // tensor-core backward (D = 64 or 128); fp32 inputs on CUDA cores
+  if (!tc_path && (dk->dtype != dq->dtype || dv->dtype != dq->dtype)) return RA_ERR_DTYPE;
+  // Set-up of the main kernel first: a set-up error returns with nothing queued.
+  BwdSm100Launch<64> lc64;
+  BwdSm100Launch<128> lc128;
+  if (tc_path) {
+    if (D == 64) RA_TRY(lc64.prepare(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv));
+    else RA_TRY(lc128.prepare(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv));
+  }
   if (meta) RA_TRY(launch_meta(mk, B, rd, meta, st));
   {
     BwdPreArgs pa;
@@ -548,8 +664,7 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
   const ProfScope prof(p, st);
   if (tc_path) {
     prof.begin();
-    const int rc = D == 64 ? launch_bwd_sm100<64>(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st)
-                           : launch_bwd_sm100<128>(q, k, v, d_o, mk, rd, meta, w, ws, dk, dv, st);
+    const int rc = D == 64 ? lc64.launch(st) : lc128.launch(st);
     prof.end();
     RA_TRY(rc);
     DqConvertArgs ca{(int)B, (int)S, (int)H, (int)D, reinterpret_cast<const float*>(ws + w.dqacc),
@@ -558,7 +673,6 @@ int ra_backward(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, cons
     dq_convert_kernel<<<(unsigned)ceil_div64(n, 256), 256, 0, st>>>(ca);
     return last_cuda();
   }
-  if (dk->dtype != dq->dtype || dv->dtype != dq->dtype) return RA_ERR_DTYPE;
   SimtBwdArgs a;
   std::memset(&a, 0, sizeof(a));
   a.rd = rd;
@@ -594,23 +708,52 @@ int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_b
   if (q_blk->ndim != 4 || k_blk->ndim != 4) return RA_ERR_SHAPE;
   const int64_t B = q_blk->shape[0], Sq = q_blk->shape[1], H = q_blk->shape[2], D = q_blk->shape[3];
   const int64_t Sk = k_blk->shape[1];
+  // A key/value block of batch 1 is shared by every query batch row (one
+  // cached prefix serving several requests); otherwise batches match.
+  const int64_t Bk = k_blk->shape[0];
   if (B < 0 || Sq < 0 || Sk < 0 || H < 0) return RA_ERR_SHAPE;
+  if (Bk != B && Bk != 1) return RA_ERR_SHAPE;
+  const bool kv_bcast = Bk == 1 && B != 1;
   RA_TRY(check_bshd(q_blk, B, Sq, H, D));
-  RA_TRY(check_bshd(k_blk, B, Sk, H, D));
-  RA_TRY(check_bshd(v_blk, B, Sk, H, D));
+  RA_TRY(check_bshd(k_blk, Bk, Sk, H, D));
+  RA_TRY(check_bshd(v_blk, Bk, Sk, H, D));
   RA_TRY(check_bshd(o_acc, B, Sq, H, D));
   RA_TRY(check_bhs(m, B, H, Sq));
   RA_TRY(check_bhs(l, B, H, Sq));
-  RA_TRY(check_bs(bias_blk, B, Sk, RA_F32));
+  RA_TRY(check_bs(bias_blk, Bk, Sk, RA_F32));
   if ((seg_q == nullptr) != (seg_k == nullptr)) return RA_ERR_NULL;
   RA_TRY(check_bs(seg_q, B, Sq, RA_I32));
-  RA_TRY(check_bs(seg_k, B, Sk, RA_I32));
+  RA_TRY(check_bs(seg_k, Bk, Sk, RA_I32));
   if (D != 64 && D != 128) return RA_ERR_UNSUPPORTED;
   const int dt = q_blk->dtype;
   if (dt != RA_BF16 && dt != RA_F32) return RA_ERR_DTYPE;
   if (!is_dtype(k_blk, dt) || !is_dtype(v_blk, dt) || o_acc->dtype != RA_F32) return RA_ERR_DTYPE;
   if (p->causal_block_size < 0 || q_off < 0 || k_off < 0) return RA_ERR_DIVISIBILITY;
+  if (m->stride[0] != l->stride[0] || m->stride[1] != l->stride[1] || m->stride[2] != l->stride[2])
+    return RA_ERR_STRIDE;
   if (B * Sq * H == 0 || Sk == 0) return RA_OK;
+  if (Sq > (int64_t(1) << 31) - kTile || Sk > (int64_t(1) << 31) - kTile) return RA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int major = bind_device(q_blk->data);
+  if (major < 0) return RA_ERR_CUDA;   // cause recorded by bind_device
+  if (dt == RA_BF16) {
+    // tensor-core step: the forward kernel in ring-step mode
+    for (const ra_tensor* t : {q_blk, k_blk, v_blk}) RA_TRY(check_tma_bf16(t));
+    RA_TRY(check_vec16(o_acc));   // the state is read and written with 16-byte vectors
+    if (major != 10) return RA_ERR_UNSUPPORTED;
+    const int32_t cbs = (int32_t)(p->causal_block_size > INT32_MAX ? INT32_MAX : p->causal_block_size);
+    auto run = [&](auto& lc) -> int {
+      RA_TRY(lc.prepare_step(q_blk, k_blk, v_blk, q_off, k_off, cbs, bias_blk, seg_q, seg_k, o_acc, m, l));
+      lc.prm.kv_bcast = kv_bcast ? 1 : 0;
+      return lc.launch(st);
+    };
+    if (D == 64) {
+      FwdSm100Launch<64, true> lc;
+      return run(lc);
+    }
+    FwdSm100Launch<128, true> lc;
+    return run(lc);
+  }
   SimtStepArgs a;
   std::memset(&a, 0, sizeof(a));
   a.B = (int)B;
@@ -625,17 +768,18 @@ int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_b
   a.q = view4(q_blk);
   a.k = view4(k_blk);
   a.v = view4(v_blk);
+  if (kv_bcast) a.k.sb = a.v.sb = 0;   // every query batch row reads key/value batch row 0
   if (seg_q) {
     a.seg_q = static_cast<const int32_t*>(seg_q->data);
     a.segq_sb = seg_q->stride[0];
     a.segq_ss = seg_q->stride[1];
     a.seg_k = static_cast<const int32_t*>(seg_k->data);
-    a.segk_sb = seg_k->stride[0];
+    a.segk_sb = kv_bcast ? 0 : seg_k->stride[0];
     a.segk_ss = seg_k->stride[1];
   }
   if (bias_blk) {
     a.bias = static_cast<const float*>(bias_blk->data);
-    a.bias_sb = bias_blk->stride[0];
+    a.bias_sb = kv_bcast ? 0 : bias_blk->stride[0];
     a.bias_ss = bias_blk->stride[1];
   }
   a.acc = static_cast<float*>(o_acc->data);
@@ -644,39 +788,22 @@ int ra_step(const ra_tensor* q_blk, const ra_tensor* k_blk, const ra_tensor* v_b
   a.acc_sh = o_acc->stride[2];
   a.m = static_cast<float*>(m->data);
   a.l = static_cast<float*>(l->data);
-  if (m->stride[0] != l->stride[0] || m->stride[1] != l->stride[1] || m->stride[2] != l->stride[2])
-    return RA_ERR_STRIDE;
   a.ml_sb = m->stride[0];
   a.ml_sh = m->stride[1];
   a.ml_ss = m->stride[2];
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   dim3 grid((unsigned)ceil_div64(Sq, kSimtRows), (unsigned)(B * H));
+  // fp32 inputs: CUDA-core step
   if (D == 64) {
     const int smem = SimtSmem<64>::BYTES;
-    if (dt == RA_BF16) {
-      if (cudaFuncSetAttribute(simt_step_kernel<64, __nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               smem) != cudaSuccess)
-        return RA_ERR_CUDA;
-      simt_step_kernel<64, __nv_bfloat16><<<grid, kSimtRows, smem, st>>>(a);
-    } else {
-      if (cudaFuncSetAttribute(simt_step_kernel<64, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-          cudaSuccess)
-        return RA_ERR_CUDA;
-      simt_step_kernel<64, float><<<grid, kSimtRows, smem, st>>>(a);
-    }
+    RA_TRY(cuda_fail(cudaFuncSetAttribute(simt_step_kernel<64, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                     "cudaFuncSetAttribute (fp32 step kernel)"));
+    simt_step_kernel<64, float><<<grid, kSimtRows, smem, st>>>(a);
   } else {
     const int smem = SimtSmem<128>::BYTES;
-    if (dt == RA_BF16) {
-      if (cudaFuncSetAttribute(simt_step_kernel<128, __nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               smem) != cudaSuccess)
-        return RA_ERR_CUDA;
-      simt_step_kernel<128, __nv_bfloat16><<<grid, kSimtRows, smem, st>>>(a);
-    } else {
-      if (cudaFuncSetAttribute(simt_step_kernel<128, float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-          cudaSuccess)
-        return RA_ERR_CUDA;
-      simt_step_kernel<128, float><<<grid, kSimtRows, smem, st>>>(a);
-    }
+    RA_TRY(cuda_fail(cudaFuncSetAttribute(simt_step_kernel<128, float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          smem),
+                     "cudaFuncSetAttribute (fp32 step kernel)"));
+    simt_step_kernel<128, float><<<grid, kSimtRows, smem, st>>>(a);
   }
   return last_cuda();
 }
@@ -703,6 +830,7 @@ int ra_finalize(const ra_tensor* o_acc, const ra_tensor* m, const ra_tensor* l, 
                  m->stride[0], m->stride[1], m->stride[2],
                  o->data, o->stride[0], o->stride[1], o->stride[2], o->dtype == RA_BF16,
                  static_cast<float*>(lse->data), lse->stride[0], lse->stride[1], lse->stride[2]};
+  if (bind_device(o_acc->data) < 0) return RA_ERR_CUDA;
   finalize_kernel<<<(unsigned)ceil_div64(n, 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return last_cuda();
 }
@@ -731,15 +859,13 @@ int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* 
               o_out->data, o_out->stride[0], o_out->stride[1], o_out->stride[2],
               static_cast<float*>(lse_out->data), lse_out->stride[0], lse_out->stride[1], lse_out->stride[2],
               dt == RA_BF16};
+  if (bind_device(o_a->data) < 0) return RA_ERR_CUDA;
   lse_merge_kernel<<<(unsigned)ceil_div64(n, 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return last_cuda();
 }
 
 int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* attention_bias,
                       const ra_tensor* segment_ids, const ra_params* p, ra_tensor* o, ra_tensor* lse, void* stream) {
-  // Device address of the static scratch, looked up once per device.
-  static std::mutex mu;
-  static void* addr[64] = {nullptr};
   if (!q || q->ndim != 4) return q ? RA_ERR_SHAPE : RA_ERR_NULL;
   if (q->shape[0] < 0 || q->shape[1] < 0 || q->shape[2] < 0 || q->shape[3] < 0) return RA_ERR_SHAPE;
   const bool need_meta = attention_bias || segment_ids;
@@ -747,15 +873,12 @@ int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v
   if (w.total > RA_STATIC_SCRATCH_BYTES) return RA_ERR_STATIC_LIMIT;
   void* scratch = nullptr;
   if (w.total > 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RA_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
-      void* ptr = nullptr;
-      if (cudaGetSymbolAddress(&ptr, g_ra_static_scratch) != cudaSuccess || !ptr) return RA_ERR_CUDA;
-      addr[dev] = ptr;
-    }
-    scratch = addr[dev];
+    // The array's device address belongs to the module loaded in the current
+    // context; it is looked up on every call (a host-side table lookup once
+    // the module is loaded), so a context that was destroyed and created
+    // again, or another context on the same device, gets its own address.
+    RA_TRY(cuda_fail(cudaGetSymbolAddress(&scratch, g_ra_static_scratch), "cudaGetSymbolAddress (static scratch)"));
+    if (!scratch) return cuda_fail(cudaErrorInvalidSymbol, "cudaGetSymbolAddress (static scratch)");
   }
   return ra_forward(q, k, v, attention_bias, segment_ids, p, o, lse, scratch, RA_STATIC_SCRATCH_BYTES, stream);
 }
@@ -855,19 +978,20 @@ int ra_train_step_host(const ra_host_step* t, const ra_tensor* attention_bias, c
   EventPool pool;
   // The copies of this step start after everything queued before it on compute_stream.
   cudaEvent_t start = pool.make();
-  if (!start || cudaEventRecord(start, sc) != cudaSuccess) return RA_ERR_CUDA;
-  if (cudaStreamWaitEvent(si, start, 0) != cudaSuccess || cudaStreamWaitEvent(so, start, 0) != cudaSuccess)
-    return RA_ERR_CUDA;
+  if (!start) return cuda_fail(cudaGetLastError(), "cudaEventCreateWithFlags");
+  RA_TRY(cuda_fail(cudaEventRecord(start, sc), "cudaEventRecord"));
+  RA_TRY(cuda_fail(cudaStreamWaitEvent(si, start, 0), "cudaStreamWaitEvent (h2d stream)"));
+  RA_TRY(cuda_fail(cudaStreamWaitEvent(so, start, 0), "cudaStreamWaitEvent (d2h stream)"));
   const int64_t hg = heads_per_group;
   for (int64_t h0 = 0; h0 < H; h0 += hg) {
     const ra_tensor* in_h[] = {&t->q, &t->k, &t->v, &t->d_o};
     const ra_tensor* in_d[] = {&t->dev_q, &t->dev_k, &t->dev_v, &t->dev_do};
     for (int i = 0; i < 4; ++i)
-      if (copy_heads(*in_d[i], *in_h[i], h0, hg, cudaMemcpyHostToDevice, si) != cudaSuccess) return RA_ERR_CUDA;
+      RA_TRY(cuda_fail(copy_heads(*in_d[i], *in_h[i], h0, hg, cudaMemcpyHostToDevice, si), "cudaMemcpy2DAsync (h2d)"));
     cudaEvent_t landed = pool.make(), done = pool.make();
-    if (!landed || !done) return RA_ERR_CUDA;
-    if (cudaEventRecord(landed, si) != cudaSuccess || cudaStreamWaitEvent(sc, landed, 0) != cudaSuccess)
-      return RA_ERR_CUDA;
+    if (!landed || !done) return cuda_fail(cudaGetLastError(), "cudaEventCreateWithFlags");
+    RA_TRY(cuda_fail(cudaEventRecord(landed, si), "cudaEventRecord"));
+    RA_TRY(cuda_fail(cudaStreamWaitEvent(sc, landed, 0), "cudaStreamWaitEvent (compute stream)"));
     ra_tensor q = head_view(t->dev_q, h0, hg), k = head_view(t->dev_k, h0, hg), v = head_view(t->dev_v, h0, hg),
               d_o = head_view(t->dev_do, h0, hg), o = head_view(t->dev_o, h0, hg),
               dq = head_view(t->dev_dq, h0, hg), dk = head_view(t->dev_dk, h0, hg),
@@ -875,24 +999,26 @@ int ra_train_step_host(const ra_host_step* t, const ra_tensor* attention_bias, c
     RA_TRY(ra_forward(&q, &k, &v, attention_bias, segment_ids, p, &o, &lse, workspace, workspace_bytes, sc));
     RA_TRY(ra_backward(&q, &k, &v, &o, &d_o, &lse, attention_bias, segment_ids, p, &dq, &dk, &dv, workspace,
                        workspace_bytes, sc));
-    if (cudaEventRecord(done, sc) != cudaSuccess || cudaStreamWaitEvent(so, done, 0) != cudaSuccess)
-      return RA_ERR_CUDA;
+    RA_TRY(cuda_fail(cudaEventRecord(done, sc), "cudaEventRecord"));
+    RA_TRY(cuda_fail(cudaStreamWaitEvent(so, done, 0), "cudaStreamWaitEvent (d2h stream)"));
     const ra_tensor* out_d[] = {&t->dev_o, &t->dev_dq, &t->dev_dk, &t->dev_dv};
     const ra_tensor* out_h[] = {&t->o, &t->dq, &t->dk, &t->dv};
     for (int i = 0; i < 4; ++i)
-      if (copy_heads(*out_h[i], *out_d[i], h0, hg, cudaMemcpyDeviceToHost, so) != cudaSuccess) return RA_ERR_CUDA;
-    if (copy_heads_bhs(t->lse, t->dev_lse, h0, hg, cudaMemcpyDeviceToHost, so) != cudaSuccess) return RA_ERR_CUDA;
+      RA_TRY(cuda_fail(copy_heads(*out_h[i], *out_d[i], h0, hg, cudaMemcpyDeviceToHost, so), "cudaMemcpy2DAsync (d2h)"));
+    RA_TRY(cuda_fail(copy_heads_bhs(t->lse, t->dev_lse, h0, hg, cudaMemcpyDeviceToHost, so), "cudaMemcpy2DAsync (d2h)"));
   }
   cudaEvent_t fin = pool.make();
-  if (!fin || cudaEventRecord(fin, so) != cudaSuccess || cudaStreamWaitEvent(sc, fin, 0) != cudaSuccess)
-    return RA_ERR_CUDA;
+  if (!fin) return cuda_fail(cudaGetLastError(), "cudaEventCreateWithFlags");
+  RA_TRY(cuda_fail(cudaEventRecord(fin, so), "cudaEventRecord"));
+  RA_TRY(cuda_fail(cudaStreamWaitEvent(sc, fin, 0), "cudaStreamWaitEvent (compute stream)"));
   return RA_OK;
 }
 
 int ra_selftest_timeout(int64_t budget_cycles, void* stream) {
   if (budget_cycles < 1000 || budget_cycles > 1000000000ll) return RA_ERR_UNSUPPORTED;
   int* ptr = nullptr;
-  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_ra_selftest_result) != cudaSuccess) return RA_ERR_CUDA;
+  RA_TRY(cuda_fail(cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_ra_selftest_result),
+                   "cudaGetSymbolAddress (self-test word)"));
   selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(budget_cycles, ptr);
   return last_cuda();
 }
@@ -936,13 +1062,15 @@ int ra_debug_set_counts(int32_t* fwd_row_counts, int32_t* bwd_col_counts) {
 #endif
 
 int ra_get_device_status(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RA_ERR_CUDA;
+  RA_TRY(cuda_fail(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)), "cudaStreamSynchronize"));
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, ra::g_ra_status, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  RA_TRY(cuda_fail(cudaMemcpyFromSymbol(&v, ra::g_ra_status, sizeof(int)), "cudaMemcpyFromSymbol (status word)"));
   const int zero = 0;
-  if (cudaMemcpyToSymbol(ra::g_ra_status, &zero, sizeof(int)) != cudaSuccess) return RA_ERR_CUDA;
+  RA_TRY(cuda_fail(cudaMemcpyToSymbol(ra::g_ra_status, &zero, sizeof(int)), "cudaMemcpyToSymbol (status word)"));
   return v;
 }
+
+const char* ra_last_error_message(void) { return t_last_error; }
 
 int64_t ra_count_visible_pairs(int64_t B, int64_t S, int64_t H, int64_t causal_block_size, const int32_t* seg_host,
                                const float* bias_host) {

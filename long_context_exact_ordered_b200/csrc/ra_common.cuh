@@ -157,12 +157,121 @@ __device__ __forceinline__ int32_t kv_iter_next_warp(KvIter& it, const RingDesc&
 }
 #endif
 
+#ifdef __CUDACC__
+// One ring step on its own ("Ring Attention技术解析" §2.2, one iteration of the
+// loop): a query block meets one visiting key/value block of Sk tokens that
+// starts at global token k_off.  StepKvIter walks that block's 128-key tiles
+// in order for the query rows [q_first, q_last] (local to the query block,
+// which starts at global token q_off), skipping tiles that causal masking
+// (global positions), disjoint segment ids or an all -inf bias hide from
+// every row.  No precomputed metadata exists for a visiting block, so a
+// converged warp computes each candidate tile's segment range and bias flags
+// itself (four keys per lane).  All functions must be called by every lane.
+struct StepKvIter {
+  int32_t tile, tile_end;
+  int32_t q_seg_min, q_seg_max;
+  const int32_t* seg_k;   // this batch row's key segment ids, or null
+  int64_t segk_ss;
+  const float* bias;      // this batch row's key bias, or null
+  int64_t bias_ss;
+  int64_t Sk;
+};
+
+// Metadata (as tile_meta_kernel writes it) of key tile t of the visiting block.
+__device__ __forceinline__ int4 step_tile_meta_warp(const StepKvIter& it, int32_t t) {
+  const int lane = threadIdx.x & 31;
+  int smin = 0x7fffffff, smax = -0x7fffffff - 1;
+  unsigned any = 0u, zero = 1u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int64_t j = (int64_t)t * kTile + lane * 4 + i;
+    if (j < it.Sk) {
+      const int s = it.seg_k ? __ldg(it.seg_k + j * it.segk_ss) : 0;
+      smin = s < smin ? s : smin;
+      smax = s > smax ? s : smax;
+      if (it.bias) {
+        const float x = __ldg(it.bias + j * it.bias_ss);
+        any |= (unsigned)(x > -INFINITY);
+        zero &= (unsigned)(x == 0.0f);
+      } else {
+        any = 1u;
+      }
+    }
+  }
+  smin = __reduce_min_sync(0xffffffffu, smin);
+  smax = __reduce_max_sync(0xffffffffu, smax);
+  any = __reduce_or_sync(0xffffffffu, any);
+  zero = __reduce_and_sync(0xffffffffu, zero);
+  return make_int4(smin, smax, (any ? kMetaAnyFinite : 0) | (zero ? kMetaAllZero : 0), 0);
+}
+
+// Segment id range of the query rows [q_first, q_last] (local, clamped to Sq).
+__device__ __forceinline__ int2 step_q_seg_range_warp(const int32_t* seg_q, int64_t segq_ss, int64_t q_first,
+                                                      int64_t q_last, int64_t Sq) {
+  const int lane = threadIdx.x & 31;
+  int smin = 0x7fffffff, smax = -0x7fffffff - 1;
+  if (q_last > Sq - 1) q_last = Sq - 1;
+  for (int64_t i = q_first + lane; i <= q_last; i += 32) {
+    const int s = __ldg(seg_q + i * segq_ss);
+    smin = s < smin ? s : smin;
+    smax = s > smax ? s : smax;
+  }
+  return make_int2(__reduce_min_sync(0xffffffffu, smin), __reduce_max_sync(0xffffffffu, smax));
+}
+
+// cbs: causal_block_size (0 = non-causal).  seg_q_b / seg_k_b: this batch
+// row's segment ids (both null without segments); bias_b: its key bias or null.
+__device__ __forceinline__ void step_iter_init_warp(StepKvIter& it, int64_t q_first, int64_t q_last, int64_t Sq,
+                                                    int64_t Sk, int64_t q_off, int64_t k_off, int32_t cbs,
+                                                    const int32_t* seg_q_b, int64_t segq_ss, const int32_t* seg_k_b,
+                                                    int64_t segk_ss, const float* bias_b, int64_t bias_ss) {
+  if (q_last > Sq - 1) q_last = Sq - 1;
+  const int32_t ntk = (int32_t)ceil_div64(Sk, kTile);
+  it.tile = 0;
+  it.tile_end = ntk;
+  if (cbs > 0) {
+    // last visible key (global) of the last query row, in this block's local terms
+    const int64_t last = ((q_off + q_last) / cbs + 1) * (int64_t)cbs - 1 - k_off;
+    const int64_t e = last < 0 ? 0 : last / kTile + 1;
+    if (e < it.tile_end) it.tile_end = (int32_t)e;
+  }
+  it.seg_k = seg_k_b;
+  it.segk_ss = segk_ss;
+  it.bias = bias_b;
+  it.bias_ss = bias_ss;
+  it.Sk = Sk;
+  it.q_seg_min = 0;
+  it.q_seg_max = 0;
+  if (seg_k_b) {
+    const int2 r = step_q_seg_range_warp(seg_q_b, segq_ss, q_first, q_last, Sq);
+    it.q_seg_min = r.x;
+    it.q_seg_max = r.y;
+  }
+}
+
+// Next visible key tile (local index) and its metadata, or -1 at the end of the block.
+__device__ __forceinline__ int32_t step_iter_next_warp(StepKvIter& it, int4& km) {
+  while (it.tile < it.tile_end) {
+    const int32_t t = it.tile++;
+    if (!it.seg_k && !it.bias) {
+      km = make_int4(0, 0, kMetaAnyFinite | kMetaAllZero, 0);
+      return t;
+    }
+    km = step_tile_meta_warp(it, t);
+    const bool seg_ok = !it.seg_k || !(km.y < it.q_seg_min || km.x > it.q_seg_max);
+    const bool bias_ok = !it.bias || (km.z & kMetaAnyFinite);
+    if (seg_ok && bias_ok) return t;
+  }
+  return -1;
+}
+#endif
+
 // Backward direction of the same ring: a key/value tile of ring block src
 // meets the query blocks (src + order[t]) mod P at steps t = 0, 1, ...
 // (rank r holds block (r - order[t]) mod P at step t).  QIter walks the
-// 64-row query tiles a key tile [k_first, k_last] must visit in that order,
+// 128-row query tiles a key tile [k_first, k_last] must visit in that order,
 // skipping tiles hidden from it by causal masking or disjoint segments.
-constexpr int kQTileBwd = 64;
+constexpr int kQTileBwd = 128;
 
 struct QIter {
   int32_t src;        // ring block of the key tile

@@ -35,6 +35,14 @@
 // in issue order.  P_q(t) is signalled per half of the keys and PV_q(t) is
 // issued in two halves, so the first half runs while the softmax still
 // computes P for the second.
+//
+// Ring-step mode (STEP = true, the per-step entry ra_step): the same kernel
+// runs one iteration of the ring loop on its own.  The query block (Sq
+// tokens starting at global token q_off) meets one visiting key/value block
+// (Sk tokens starting at k_off); masks use global positions; the block's
+// tiles are visited in order (StepKvIter); and the epilogue merges the
+// block's partial (reference max, sum, unnormalised O) into the caller's
+// running fp32 state (m, l, o_acc) instead of writing O and LSE.
 #pragma once
 
 #include <cuda.h>
@@ -96,11 +104,59 @@ struct FwdParams {
   int64_t bias_sb, bias_ss;
   const int4* meta;        // [B, ntiles] or null
   int32_t* dbg_count;      // RA_DEBUG_COUNT builds: visible keys per query row, [B, H, S]
+  // Ring-step mode only (rd.S is then Sq, `seg` the query block's ids and
+  // `bias` the visiting keys' bias [B, Sk]).
+  int64_t Sk, q_off, k_off;
+  const int32_t* seg_k;    // [B, Sk] visiting keys' segment ids, or null
+  int64_t segk_sb, segk_ss;
+  float* acc;              // [B, Sq, H, D] fp32 running unnormalised output
+  int64_t acc_sb, acc_ss, acc_sh;
+  float* m_state;          // [B, H, Sq] running max (natural-log units)
+  float* l_state;          // [B, H, Sq] running sum
+  int64_t ml_sb, ml_sh, ml_ss;
+  int32_t kv_bcast;        // 1: the key/value block (and its bias / segment ids) has batch 1, shared by every query row b
+};
+
+// The key/value tiles a pair of query tiles visits: the whole ring
+// (KvIter, tile metadata precomputed) or, in ring-step mode, the visiting
+// block (StepKvIter, metadata computed on the fly).  Every lane of a warp
+// calls these.
+template <bool STEP>
+struct FwdTiles;
+
+template <>
+struct FwdTiles<false> {
+  KvIter it;
+  const int4* meta_b;
+  __device__ __forceinline__ void init(const FwdParams& p, int, int64_t q0, const int4* mb, bool use_seg,
+                                       bool use_bias) {
+    meta_b = mb;
+    kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, mb, use_seg, use_bias);
+  }
+  __device__ __forceinline__ int32_t next(const FwdParams& p) { return kv_iter_next_warp(it, p.rd); }
+  __device__ __forceinline__ int4 meta(int32_t t) const {
+    return meta_b ? load_meta(meta_b + t) : make_int4(0, 0, kMetaAnyFinite | kMetaAllZero, 0);
+  }
+};
+
+template <>
+struct FwdTiles<true> {
+  StepKvIter it;
+  int4 km;
+  __device__ __forceinline__ void init(const FwdParams& p, int b, int64_t q0, const int4*, bool use_seg,
+                                       bool use_bias) {
+    step_iter_init_warp(it, q0, q0 + 2 * kTile - 1, p.rd.S, p.Sk, p.q_off, p.k_off, p.rd.cbs,
+                        use_seg ? p.seg + b * p.seg_sb : nullptr, p.seg_ss,
+                        use_seg ? p.seg_k + (p.kv_bcast ? 0 : b) * p.segk_sb : nullptr, p.segk_ss,
+                        use_bias ? p.bias + (p.kv_bcast ? 0 : b) * p.bias_sb : nullptr, p.bias_ss);
+  }
+  __device__ __forceinline__ int32_t next(const FwdParams&) { return step_iter_next_warp(it, km); }
+  __device__ __forceinline__ int4 meta(int32_t) const { return km; }
 };
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
-template <int D>
+template <int D, bool STEP>
 __global__ void __launch_bounds__(384, 1)
     ra_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ FwdParams p) {
@@ -117,8 +173,10 @@ __global__ void __launch_bounds__(384, 1)
   const int pair = p.npairs - 1 - unit % p.npairs;
   const int bh = unit / p.npairs;
   const int b = bh / p.H, h = bh % p.H;
+  const int bk = (STEP && p.kv_bcast) ? 0 : b;   // batch row of the key/value side
   const int64_t q0 = (int64_t)pair * 2 * kTile;
-  const int64_t S = p.rd.S;
+  const int64_t S = p.rd.S;                   // query rows (Sq in ring-step mode)
+  const int64_t Sk = STEP ? p.Sk : S;         // key rows
 
   auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::OFF_MISC);
@@ -168,18 +226,18 @@ __global__ void __launch_bounds__(384, 1)
                         (int)(q0 + qt * kTile), b);
       }
       __syncwarp();
-      KvIter it;
-      kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
+      FwdTiles<STEP> tiles;
+      tiles.init(p, b, q0, meta_b, use_seg, use_bias);
       const uint64_t pol = l2_policy_evict_last();   // K/V tiles are re-read by every query pair of the head
       int nk = 0, nv = 0;   // K / V tiles issued
-      for (int32_t t = kv_iter_next_warp(it, p.rd); t >= 0; t = kv_iter_next_warp(it, p.rd)) {
+      for (int32_t t = tiles.next(p); t >= 0; t = tiles.next(p)) {
         const int ks = nk % L::KS, vs = nv % L::VS;
         if (nk >= L::KS && !ra_wait_warp(bar(L::B_KEMPTY + ks), ((nk / L::KS) & 1) ^ 1, abort_flag)) break;
         if (elect_one()) {
           mbar_arrive_expect_tx(bar(L::B_KFULL + ks), L::TILE_BYTES);
           for (int c = 0; c < L::KCH; ++c)
             tma_load_4d_hint(sbase + L::OFF_K + ks * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_k, bar(L::B_KFULL + ks),
-                             c * 64, h, t * kTile, b, pol);
+                             c * 64, h, t * kTile, bk, pol);
         }
         __syncwarp();
         ++nk;
@@ -188,7 +246,7 @@ __global__ void __launch_bounds__(384, 1)
           mbar_arrive_expect_tx(bar(L::B_VFULL + vs), L::TILE_BYTES);
           for (int c = 0; c < L::KCH; ++c)
             tma_load_4d_hint(sbase + L::OFF_V + vs * L::TILE_BYTES + c * L::CHUNK_BYTES, &tm_v, bar(L::B_VFULL + vs),
-                             c * 64, h, t * kTile, b, pol);
+                             c * 64, h, t * kTile, bk, pol);
         }
         __syncwarp();
         ++nv;
@@ -226,9 +284,9 @@ __global__ void __launch_bounds__(384, 1)
                    (acc || k > 0) ? 1u : 0u);
         }
       };
-      KvIter it;
-      kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
-      int32_t t = kv_iter_next_warp(it, p.rd);
+      FwdTiles<STEP> tiles;
+      tiles.init(p, b, q0, meta_b, use_seg, use_bias);
+      int32_t t = tiles.next(p);
       bool ok = ra_wait_warp(bar(L::B_Q), 0, abort_flag);
       if (ok && t >= 0) {
         ok = ra_wait_warp(bar(L::B_KFULL + 0), 0, abort_flag);
@@ -241,7 +299,7 @@ __global__ void __launch_bounds__(384, 1)
           mma_commit_w(bar(L::B_KEMPTY + 0));
         }
         for (int n = 0; ok; ++n) {
-          const int32_t tn = kv_iter_next_warp(it, p.rd);
+          const int32_t tn = tiles.next(p);
           const bool last = tn < 0;
           const int vs = n % L::VS, ks1 = (n + 1) % L::KS;
           const uint32_t ph = n & 1;
@@ -301,27 +359,41 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO_row = tmem + lane_off + (qt ? L::COL_O1 : L::COL_O0);
     const int64_t qrow_c = qrow < S ? qrow : S - 1;
     const int my_seg = use_seg ? p.seg[b * p.seg_sb + qrow_c * p.seg_ss] : 0;
-    const int q_tile_idx = (int)(q_first / kTile);
-    const int4 qm = (meta_b && q_tile_idx < p.rd.ntiles) ? load_meta(meta_b + q_tile_idx) : make_int4(0, 0, 3, 0);
+    // key-side segment ids (the visiting block's in ring-step mode)
+    const int32_t* segk = STEP ? p.seg_k : p.seg;
+    const int64_t segk_sb = STEP ? p.segk_sb : p.seg_sb, segk_ss = STEP ? p.segk_ss : p.seg_ss;
+    int4 qm = make_int4(0, 0, kMetaAnyFinite | kMetaAllZero, 0);
+    if constexpr (STEP) {
+      if (use_seg) {
+        const int2 r = step_q_seg_range_warp(p.seg + b * p.seg_sb, p.seg_ss, q_first, q_first + kTile - 1, S);
+        qm.x = r.x;
+        qm.y = r.y;
+      }
+    } else {
+      const int q_tile_idx = (int)(q_first / kTile);
+      if (meta_b && q_tile_idx < p.rd.ntiles) qm = load_meta(meta_b + q_tile_idx);
+    }
     const int32_t cbs = p.rd.cbs;
-    const int64_t causal_jmax = cbs > 0 ? (qrow / cbs + 1) * (int64_t)cbs - 1 : S - 1;
+    // Masks compare global positions; keys are indexed locally from k_base.
+    const int64_t q_base = STEP ? p.q_off : 0, k_base = STEP ? p.k_off : 0;
+    const int64_t causal_jmax = cbs > 0 ? ((q_base + qrow) / cbs + 1) * (int64_t)cbs - 1 - k_base : Sk - 1;
     // Per-tile mask test without divisions: a KV tile needs the per-element
     // mask iff it reaches past the causal block of the tile's first query
-    // (k_last > q_blk_end), runs past S, or mixes segment ids.
-    const int64_t q_blk_end = cbs > 0 ? (q_first / cbs + 1) * (int64_t)cbs - 1 : INT64_MAX;
+    // (k_last > q_blk_end), runs past the last key, or mixes segment ids.
+    const int64_t q_blk_end = cbs > 0 ? ((q_base + q_first) / cbs + 1) * (int64_t)cbs - 1 - k_base : INT64_MAX;
     const bool q_seg_uniform = qm.x == qm.y;
 
-    KvIter it;
-    kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, meta_b, use_seg, use_bias);
+    FwdTiles<STEP> tiles;
+    tiles.init(p, b, q0, meta_b, use_seg, use_bias);
     float m_ref = -INFINITY, l = 0.f;
 #ifdef RA_DEBUG_COUNT
     int dbg_vis = 0;
 #endif
     int n = 0;
     bool ok = true;
-    for (int32_t t = kv_iter_next_warp(it, p.rd); t >= 0; t = kv_iter_next_warp(it, p.rd), ++n) {
+    for (int32_t t = tiles.next(p); t >= 0; t = tiles.next(p), ++n) {
       // the tile's metadata load is issued before the wait, so it lands while S is computed
-      const int4 km = meta_b ? load_meta(meta_b + t) : make_int4(0, 0, 3, 0);
+      const int4 km = tiles.meta(t);
       if (!(ok = ra_wait_warp(bar(L::B_SFULL + qt), n & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t sr[128];
@@ -340,12 +412,12 @@ __global__ void __launch_bounds__(384, 1)
       // (the empty asm keeps the compiler from hoisting all 128 and spilling).
       const bool has_bias = use_bias && !(km.z & kMetaAllZero);
       if (has_bias) {
-        const float* bp = p.bias + b * p.bias_sb;
+        const float* bp = p.bias + bk * p.bias_sb;
 #pragma unroll
         for (int c0 = 0; c0 < 128; c0 += 32) {
 #pragma unroll
           for (int c = c0; c < c0 + 32; ++c) {
-            const int64_t j = k0 + c < S ? k0 + c : S - 1;
+            const int64_t j = k0 + c < Sk ? k0 + c : Sk - 1;
             x[c] = fmaf(x[c], p.scale_log2, __ldg(bp + j * p.bias_ss) * kLog2e);
           }
           asm volatile("" ::: "memory");
@@ -353,22 +425,22 @@ __global__ void __launch_bounds__(384, 1)
       }
       // per-element mask on diagonal / ragged / mixed-segment tiles
       const int64_t k_last = k0 + kTile - 1;
-      const bool need_mask = k_last > S - 1 || k_last > q_blk_end ||
+      const bool need_mask = k_last > Sk - 1 || k_last > q_blk_end ||
                              (use_seg && !(q_seg_uniform && km.x == km.y && qm.x == km.x));
       if (need_mask) {
-        int64_t jmax = causal_jmax < S - 1 ? causal_jmax : S - 1;
+        int64_t jmax = causal_jmax < Sk - 1 ? causal_jmax : Sk - 1;
         const int64_t lim64 = jmax - k0;
         const int lim = lim64 < -1 ? -1 : (lim64 > 127 ? 127 : (int)lim64);
         uint32_t vb[4] = {~0u, ~0u, ~0u, ~0u};   // segment match bits, 32 keys per word
         if (use_seg) {
-          const int32_t* sp = p.seg + b * p.seg_sb;
+          const int32_t* sp = segk + bk * segk_sb;
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
             uint32_t bits = 0;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-              const int64_t j = k0 + 32 * w + c < S ? k0 + 32 * w + c : S - 1;
-              bits |= (uint32_t)(__ldg(sp + j * p.seg_ss) == my_seg) << c;
+              const int64_t j = k0 + 32 * w + c < Sk ? k0 + 32 * w + c : Sk - 1;
+              bits |= (uint32_t)(__ldg(sp + j * segk_ss) == my_seg) << c;
             }
             vb[w] = bits;
             asm volatile("" ::: "memory");
@@ -448,39 +520,86 @@ __global__ void __launch_bounds__(384, 1)
     if (ok && n > 0) ok = ra_wait_warp(bar(L::B_PVDONE + qt), (n - 1) & 1, abort_flag);
     n = __shfl_sync(0xffffffffu, n, 0);   // warp-uniform (lanes agree unless a wait gave up)
     tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16* op = p.o + b * p.o_sb + qrow_c * p.o_ss + h * p.o_sh;
+    if constexpr (STEP) {
+      // Merge this block's partial (reference max m_ref in log2 units, sum l,
+      // O in TMEM, both relative to 2^m_ref) into the caller's running state
+      // (m in natural-log units, l, o_acc relative to e^m):
+      //   m' = max(m, m_blk), o_acc' = e^(m - m') o_acc + e^(m_blk - m') O, l' likewise.
+      const int64_t mi = b * p.ml_sb + h * p.ml_sh + qrow_c * p.ml_ss;
+      const float m_in = p.m_state[mi], l_in = p.l_state[mi];
+      const float m_blk = (n > 0 && m_ref != -INFINITY) ? m_ref * kLn2 : -INFINITY;
+      const float m_new = fmaxf(m_in, m_blk);
+      const bool write = qrow < S && ok && m_new != -INFINITY;
+      const float a_in = m_in == -INFINITY ? 0.f : expf(m_in - m_new);
+      const float a_blk = m_blk == -INFINITY ? 0.f : expf(m_blk - m_new);
+      float* ap = p.acc + b * p.acc_sb + qrow_c * p.acc_ss + h * p.acc_sh;
 #pragma unroll
-    for (int c = 0; c < D; c += 32) {
-      uint32_t orow[32];
-      if (n > 0) {
-        tmem_ld32(tO_row + c, orow);
-        tmem_ld_wait();
-      }
-      uint32_t pkd[16];
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float a0 = 0.f, a1 = 0.f;
+      for (int c = 0; c < D; c += 32) {
+        uint32_t orow[32];
         if (n > 0) {
-          reg_fence(orow[e]);
-          reg_fence(orow[e + 1]);
-          a0 = __uint_as_float(orow[e]) * inv;
-          a1 = __uint_as_float(orow[e + 1]) * inv;
+          tmem_ld32(tO_row + c, orow);
+          tmem_ld_wait();
         }
-        pkd[e >> 1] = pack_bf16x2(a0, a1);
-      }
-      if (qrow < S && ok) {
-        uint4* dst = reinterpret_cast<uint4*>(op + c);
+        if (write) {
+          float4* a4 = reinterpret_cast<float4*>(ap + c);
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+          for (int v4 = 0; v4 < 8; ++v4) {
+            float o4[4] = {0.f, 0.f, 0.f, 0.f};
+            if (n > 0) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                reg_fence(orow[4 * v4 + e]);
+                o4[e] = __uint_as_float(orow[4 * v4 + e]);
+              }
+            }
+            float4 x = a4[v4];
+            x.x = fmaf(a_in, x.x, a_blk * o4[0]);
+            x.y = fmaf(a_in, x.y, a_blk * o4[1]);
+            x.z = fmaf(a_in, x.z, a_blk * o4[2]);
+            x.w = fmaf(a_in, x.w, a_blk * o4[3]);
+            a4[v4] = x;
+          }
+        }
       }
-    }
-    if (qrow < S && ok)
-      p.lse[b * p.lse_sb + h * p.lse_sh + qrow * p.lse_ss] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+      if (write) {
+        p.m_state[mi] = m_new;
+        p.l_state[mi] = fmaf(a_in, l_in, a_blk * l);
+      }
+    } else {
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* op = p.o + b * p.o_sb + qrow_c * p.o_ss + h * p.o_sh;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t orow[32];
+        if (n > 0) {
+          tmem_ld32(tO_row + c, orow);
+          tmem_ld_wait();
+        }
+        uint32_t pkd[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float a0 = 0.f, a1 = 0.f;
+          if (n > 0) {
+            reg_fence(orow[e]);
+            reg_fence(orow[e + 1]);
+            a0 = __uint_as_float(orow[e]) * inv;
+            a1 = __uint_as_float(orow[e + 1]) * inv;
+          }
+          pkd[e >> 1] = pack_bf16x2(a0, a1);
+        }
+        if (qrow < S && ok) {
+          uint4* dst = reinterpret_cast<uint4*>(op + c);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pkd[4 * v4], pkd[4 * v4 + 1], pkd[4 * v4 + 2], pkd[4 * v4 + 3]);
+        }
+      }
+      if (qrow < S && ok)
+        p.lse[b * p.lse_sb + h * p.lse_sh + qrow * p.lse_ss] = l > 0.f ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
 #ifdef RA_DEBUG_COUNT
-    if (qrow < S && ok && p.dbg_count) p.dbg_count[((int64_t)b * p.H + h) * S + qrow] = dbg_vis;
+      if (qrow < S && ok && p.dbg_count) p.dbg_count[((int64_t)b * p.H + h) * S + qrow] = dbg_vis;
 #endif
+    }
   }
 
   // ------------------------------------------------------------ teardown

@@ -25,6 +25,8 @@ Modules
                analytic backward, float64 numpy (the oracle proper).
 ``loops``      the same definition as pure-Python loops for tiny inputs
                (an independent restatement used to pin ``attention``).
+``feedforward`` the blockwise feed-forward network (SwiGLU) exported next
+               to ``ringattention``.
 ``ring``       the ring-blockwise path (P virtual ranks, chunked online
                softmax, log-sum-exp merge): a second, independent route to
                the same numbers, used only by the oracle's self-tests.
@@ -37,6 +39,7 @@ from .attention import (  # noqa: F401
     attention_backward,
     attention_forward,
     attention_rows,
+    backward_term_magnitudes,
     causal_ok,
     head_backward_cols,
     visible_count_cols,
@@ -44,4 +47,5 @@ from .attention import (  # noqa: F401
     visible_mask,
     visible_pairs_total,
 )
+from .feedforward import blockwise_feedforward, silu  # noqa: F401
 from .ring import finalize, lse_merge, online_step, ring_blockwise_reference  # noqa: F401

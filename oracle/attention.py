@@ -281,6 +281,52 @@ def attention_backward_rows(q, k, v, do, samples, attention_bias=None, segment_i
     return dq
 
 
+def backward_term_magnitudes(q, k, v, do, attention_bias=None, segment_ids=None, causal_block_size=None,
+                             o=None, lse=None):
+    """The sums of the backward's terms taken in absolute value, float64.
+
+    Returns (mag_dq, mag_dk, mag_dv) [B,S,H,D]:
+
+        mag_dq_i = scale sum_j |dS_ij| |k_j|,   mag_dk_j = scale sum_i |dS_ij| |q_i|,
+        mag_dv_j = sum_i P_ij |dO_i|            (|.| element-wise on vectors)
+
+    with P and dS the same quantities as in ``attention_backward``.  They are
+    not part of the method: they bound how far a backward may move when its
+    product operands dS and P are rounded, element by element, with relative
+    error at most u before the sums (each term moves by at most u times its
+    magnitude), which is how the tests hold a bf16 tensor-core backward to the
+    exact gradients.  ``o`` / ``lse`` as in ``attention_backward``.
+    """
+    q = np.asarray(q)
+    B, S, H, D = q.shape
+    scale = 1.0 / math.sqrt(D)
+    if o is None or lse is None:
+        o, lse = attention_forward(q, k, v, attention_bias, segment_ids, causal_block_size)
+    mq = np.zeros((B, S, H, D), dtype=np.float64)
+    mk = np.zeros((B, S, H, D), dtype=np.float64)
+    mv = np.zeros((B, S, H, D), dtype=np.float64)
+    for b in range(B):
+        seg_b = None if segment_ids is None else np.asarray(segment_ids)[b]
+        bias_b = None if attention_bias is None else _f64(attention_bias)[b]
+        for h in range(H):
+            qh, kh, vh, doh = _f64(q[b, :, h]), _f64(k[b, :, h]), _f64(v[b, :, h]), _f64(do[b, :, h])
+            oh, lse_h = _f64(o[b, :, h]), _f64(lse[b, h])
+            for a, e in _row_chunks(S, S):
+                rows = np.arange(a, e)
+                vis = visible_mask(rows, S, causal_block_size, seg_b, bias_b)
+                s = scale * (qh[a:e] @ kh.T)
+                if bias_b is not None:
+                    s = s + np.where(np.isfinite(bias_b), bias_b, 0.0)[None, :]
+                has = np.isfinite(lse_h[a:e])
+                P = np.where(vis & has[:, None], np.exp(s - np.where(has, lse_h[a:e], 0.0)[:, None]), 0.0)
+                Dl = np.sum(doh[a:e] * oh[a:e], axis=1)
+                dS = np.abs(P * (doh[a:e] @ vh.T - Dl[:, None]))
+                mq[b, a:e, h] = scale * (dS @ np.abs(kh))
+                mk[b, :, h] += scale * (dS.T @ np.abs(qh[a:e]))
+                mv[b, :, h] += P.T @ np.abs(doh[a:e])
+    return mq, mk, mv
+
+
 def visible_count_rows(rows, S, causal_block_size=None, seg_b=None, bias_b=None):
     """Exact integer number of visible keys for each query row of one batch."""
     rows = np.asarray(rows, dtype=np.int64)

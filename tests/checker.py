@@ -10,6 +10,16 @@ Tolerances (stated once, used by every parity test):
   error is reported next to it.  The mean-abs bound is applied raw.
 * fp32 outputs: max-abs error <= 1e-5 (raw).
 * integer outputs (counts, masks): bit-exact.
+* bf16 gradients of inputs with a random additive bias: the tensor-core
+  backward rounds its product operands dS and P to bf16 (relative error at
+  most u = 2^-8 each) before the fp32 sums dQ = scale dS K, dK = scale dS^T Q,
+  dV = P^T dO.  Each term then moves by at most u times its magnitude, so a
+  correct backward can differ from the exact gradient by up to
+  u * sum|terms| (oracle.backward_term_magnitudes), plus the fp32 sums'
+  own n * 2^-24 relative error.  When a few keys carry most of the attention
+  that bound exceeds 1e-2.  For those cases an element passes when its
+  excess over half a bf16 ulp is within max(1e-2, that bound); the mean-abs
+  bound stays 1e-3.  Every other case uses the plain bf16 rule.
 """
 
 from __future__ import annotations
@@ -21,6 +31,15 @@ import numpy as np
 BF16_MAX_ABS = 1e-2
 BF16_MEAN_ABS = 1e-3
 F32_MAX_ABS = 1e-5
+BF16_UNIT_ROUNDOFF = 2.0 ** -8    # round-to-nearest with an 8-bit significand
+F32_UNIT_ROUNDOFF = 2.0 ** -24
+
+
+def operand_rounding_bound(magnitude, n_terms):
+    """Largest change of a sum of n_terms products when one factor of every
+    term is rounded to bf16 and the sum is formed in fp32: (u_bf16 + n *
+    u_f32) * sum|terms|, with ``magnitude`` = sum|terms| element-wise."""
+    return (BF16_UNIT_ROUNDOFF + n_terms * F32_UNIT_ROUNDOFF) * np.asarray(magnitude, dtype=np.float64)
 
 
 def bf16_half_ulp(x):
@@ -45,8 +64,12 @@ class Cmp:
                 f"max_excess={self.max_excess:.3e} mean_abs={self.mean_abs:.3e} n={self.n}")
 
 
-def compare(gpu, ref, kind="bf16", max_abs=None, mean_abs=None) -> Cmp:
-    """Compare arrays; ``kind`` is "bf16" (half-ulp excess rule) or "f32"."""
+def compare(gpu, ref, kind="bf16", max_abs=None, mean_abs=None, rounding_bound=None) -> Cmp:
+    """Compare arrays; ``kind`` is "bf16" (half-ulp excess rule) or "f32".
+
+    ``rounding_bound`` (bf16 only): an array like ``ref`` from
+    ``operand_rounding_bound``; the allowed excess of each element is then
+    max(max_abs, rounding_bound) instead of max_abs."""
     g = np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (g.shape, r.shape)
@@ -60,9 +83,15 @@ def compare(gpu, ref, kind="bf16", max_abs=None, mean_abs=None) -> Cmp:
         lim = BF16_MAX_ABS if max_abs is None else max_abs
         mlim = BF16_MEAN_ABS if mean_abs is None else mean_abs
         excess = np.maximum(0.0, err - np.where(np.isfinite(r), bf16_half_ulp(r), 0.0))
+        if rounding_bound is None:
+            allowed = lim
+            rule = f"bf16(excess<={lim:g}, mean<={mlim:g})"
+        else:
+            allowed = np.maximum(lim, np.asarray(rounding_bound, dtype=np.float64))
+            rule = f"bf16(excess<=max({lim:g}, operand rounding bound), mean<={mlim:g})"
+        over = excess - allowed
         mex = float(excess.max()) if n else 0.0
-        ok = mex <= lim and mean <= mlim
-        rule = f"bf16(excess<={lim:g}, mean<={mlim:g})"
+        ok = (float(over.max()) <= 0.0 if n else True) and mean <= mlim
     else:
         lim = F32_MAX_ABS if max_abs is None else max_abs
         mex = mx

@@ -3,14 +3,18 @@
 The backward receives the forward output as stored (bf16 for bf16 inputs)
 and forms Delta_i = <dO_i, o_i> from it, so the oracle's reference gradient
 takes Delta from its own float64 output rounded (nearest even) to the input
-dtype.  Random additive biases here are N(0, 0.5^2) (plus masked keys): with
-N(0, 1) biases a few keys absorb most of the attention of many rows, and the
-bf16 rounding of P in dV = P^T dO alone then exceeds 1e-2 absolute.
+dtype.
 
 dQ, dK, dV: bf16 outputs use the bf16 rule of checker.py (max-abs excess over
-half a bf16 ulp <= 1e-2, mean-abs <= 1e-3); fp32 gradient outputs of bf16
-inputs use the raw max-abs 1e-2 / mean-abs 1e-3; fp32 inputs (CUDA-core path)
-use max-abs 1e-4 (gradients sum many more terms than the forward).
+half a bf16 ulp <= 1e-2, mean-abs <= 1e-3).  Cases with a random additive
+bias draw it from N(0, 1) with a fifth of the keys masked (-inf): a few keys
+then carry most of the attention of many rows, and the bf16 rounding of the
+P and dS operands can move a gradient element by more than 1e-2; those cases
+allow each element the exact bound of that rounding,
+max(1e-2, operand_rounding_bound(backward_term_magnitudes)) (checker.py).
+fp32 gradient outputs of bf16 inputs use the raw max-abs 1e-2 / mean-abs
+1e-3; fp32 inputs (CUDA-core path) use max-abs 1e-4 (gradients sum many more
+terms than the forward).
 """
 
 from __future__ import annotations
@@ -21,7 +25,7 @@ import torch
 
 import oracle
 import workloads as W
-from checker import compare
+from checker import compare, operand_rounding_bound
 from gpu_util import gather_rows, oracle_rows, to64, to_np
 
 pytestmark = pytest.mark.gpu
@@ -47,7 +51,7 @@ def make(D, S, P, c, segments, bias, B, H, dtype="bf16", seed=21):
     inp = W.make_inputs(w, dev())
     if bias == "neginf":
         g = torch.Generator(device="cpu").manual_seed(seed + 1)
-        b = 0.5 * torch.randn((B, S), generator=g)
+        b = torch.randn((B, S), generator=g)
         b[:, torch.randint(0, S, (S // 5,), generator=g)] = float("-inf")
         inp["bias"] = b.to(dev())
     return w, inp
@@ -67,11 +71,19 @@ def stored(o64, dtype):
     return torch.from_numpy(o64).to(dtype).double().numpy()
 
 
-def oracle_grads(inp, c):
+def oracle_grads(inp, c, bounds=False):
+    """Oracle gradients (dq, dk, dv); with ``bounds``, also the per-element
+    operand rounding bounds of the three gradients (checker.py)."""
     args = [to64(inp[n]) for n in ("q", "k", "v", "do")]
     bias, seg = to64(inp["bias"]), to_np(inp["seg"])
     o, lse = oracle.attention_forward(*args[:3], bias, seg, c)
-    return oracle.attention_backward(*args, bias, seg, c, o=stored(o, inp["q"].dtype), lse=lse)
+    o_st = stored(o, inp["q"].dtype)
+    grads = oracle.attention_backward(*args, bias, seg, c, o=o_st, lse=lse)
+    if not bounds:
+        return grads
+    S = args[0].shape[1]
+    mags = oracle.backward_term_magnitudes(*args, bias, seg, c, o=o_st, lse=lse)
+    return grads, tuple(operand_rounding_bound(m, S) for m in mags)
 
 
 CASES = [
@@ -92,9 +104,13 @@ CASES = [
 def test_bf16_backward_full_parity(case):
     w, inp = make(*case)
     o, lse, (dq, dk, dv) = run_both(w, inp)
-    rq, rk, rv = oracle_grads(inp, w.causal_block_size)
-    for name, g, r in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
-        res = compare(to64(g), r, "bf16")
+    if inp["bias"] is None:
+        rq, rk, rv = oracle_grads(inp, w.causal_block_size)
+        bq = bk = bv = None
+    else:
+        (rq, rk, rv), (bq, bk, bv) = oracle_grads(inp, w.causal_block_size, bounds=True)
+    for name, g, r, bnd in (("dq", dq, rq, bq), ("dk", dk, rk, bk), ("dv", dv, rv, bv)):
+        res = compare(to64(g), r, "bf16", rounding_bound=bnd)
         assert res.ok, f"{name}: {res}"
 
 
@@ -165,13 +181,14 @@ def test_autograd_function_matches_explicit_calls():
     assert torch.equal(k.grad, dk) and torch.equal(v.grad, dv)
 
 
-def _rows_grad_stored(qh, kh, vh, doh, sub):
-    """dQ rows with Delta from the stored (bf16-rounded) output rows."""
+def _rows_grad_stored(qh, kh, vh, doh, sub, seg_b=None):
+    """dQ rows with Delta from the stored (bf16-rounded) output rows.  ``seg_b``:
+    the batch row's segment ids [S] or None."""
     from oracle.attention import _head_backward
     rows = sub[:, 2]
-    o_r, lse_r = oracle.attention_rows(qh, kh, vh, sub, None, None, 1)
+    o_r, lse_r = oracle.attention_rows(qh, kh, vh, sub, None, None if seg_b is None else seg_b[None], 1)
     dq, _, _ = _head_backward(qh[0, rows, 0], kh[0, :, 0], vh[0, :, 0], doh[0, rows, 0],
-                              stored(o_r, torch.bfloat16), lse_r, rows, 1, None, None, want_dkdv=False)
+                              stored(o_r, torch.bfloat16), lse_r, rows, 1, seg_b, None, want_dkdv=False)
     return dq
 
 
@@ -207,16 +224,18 @@ def test_config_causal64k_fwd_bwd():
     np.testing.assert_allclose(to64(dv).sum(axis=1), to64(inp["do"]).sum(axis=1), atol=tol)
 
 
-@pytest.mark.slow
-def test_config_causal128k_fwd_bwd():
-    """The bench's workload at full size, in the bench's launch configuration
-    (128K causal, B=1, H=32, D=128, P=8, chunks 512): O and LSE on 4096 sampled
-    rows, dQ on the same rows, dK / dV on 512 sampled keys of one seeded head
-    (including every ring-block boundary), and the invariants on all heads."""
-    w = W.WORKLOADS["causal128k"]
-    inp = W.make_inputs(w, dev())
+def _full_size_fwd_bwd(name):
+    """A 128K workload at full size, in the bench's launch configuration (B=1,
+    H=32, D=128, P=8, chunks 512): O and LSE on 4096 sampled rows, dQ on the
+    same rows, dK / dV on 512 sampled keys of one seeded head (including every
+    ring-block boundary and, with packed documents, every document start), and
+    the invariants on all heads."""
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w, dev(), with_grad_output=True)
     o, lse, (dq, dk, dv) = run_both(w, inp)
-    samples = W.sample_rows(w, None, n=4096)
+    seg = None if inp["seg"] is None else to_np(inp["seg"])
+    seg_b = None if seg is None else seg[0]
+    samples = W.sample_rows(w, seg, n=4096)
     sel = (torch.as_tensor(samples[:, 0]), torch.as_tensor(samples[:, 2]), torch.as_tensor(samples[:, 1]))
     # forward rows (one head's K / V on the host at a time)
     ro, rl = oracle_rows(inp, samples, 1)
@@ -232,21 +251,40 @@ def test_config_causal128k_fwd_bwd():
         rows = samples[idx, 2]
         sub = np.stack([np.zeros_like(rows), np.zeros_like(rows), rows], axis=1)
         qh, kh, vh, doh = (to64(inp[n][0, :, int(h)].contiguous())[None, :, None, :] for n in ("q", "k", "v", "do"))
-        want[idx] = _rows_grad_stored(qh, kh, vh, doh, sub)
+        want[idx] = _rows_grad_stored(qh, kh, vh, doh, sub, seg_b)
     res = compare(got, want, "bf16")
     assert res.ok, f"dq rows: {res}"
     # dK / dV on sampled keys of one head (its full forward gives every row's lse and stored o)
     rng = np.random.default_rng(w.seed + 9)
     h = int(rng.integers(0, w.H))
     blk = w.S // w.P
-    edges = np.concatenate([np.arange(w.P) * blk, np.arange(1, w.P + 1) * blk - 1])
-    cols = np.unique(np.concatenate([edges, rng.choice(w.S, size=512 - len(edges), replace=False)]))
+    must = [np.arange(w.P) * blk, np.arange(1, w.P + 1) * blk - 1]
+    if seg_b is not None:
+        must.append(np.nonzero(np.r_[True, seg_b[1:] != seg_b[:-1]])[0])
+    must = np.unique(np.concatenate(must))
+    cols = np.unique(np.concatenate([must, rng.choice(w.S, size=512 - len(must), replace=False)]))
     qh, kh, vh, doh = (to64(inp[n][0, :, h].contiguous()) for n in ("q", "k", "v", "do"))
-    o_h, l_h = oracle.attention_forward(qh[None, :, None], kh[None, :, None], vh[None, :, None], None, None, 1)
-    rk, rv = oracle.head_backward_cols(qh, kh, vh, doh, stored(o_h, torch.bfloat16)[0, :, 0], l_h[0, 0], cols, 1)
-    assert compare(to64(dk[0, torch.as_tensor(cols), h]), rk, "bf16").ok
-    assert compare(to64(dv[0, torch.as_tensor(cols), h]), rv, "bf16").ok
+    sg = None if seg is None else seg[:1]
+    o_h, l_h = oracle.attention_forward(qh[None, :, None], kh[None, :, None], vh[None, :, None], None, sg, 1)
+    rk, rv = oracle.head_backward_cols(qh, kh, vh, doh, stored(o_h, torch.bfloat16)[0, :, 0], l_h[0, 0], cols, 1,
+                                       seg_b)
+    res = compare(to64(dk[0, torch.as_tensor(cols), h]), rk, "bf16")
+    assert res.ok, f"dk cols: {res}"
+    res = compare(to64(dv[0, torch.as_tensor(cols), h]), rv, "bf16")
+    assert res.ok, f"dv cols: {res}"
     tol = 1e-2 * np.sqrt(w.S)
     sum64 = lambda t: t.double().sum(dim=1).cpu().numpy()    # sums over tokens, in float64 on the device
     np.testing.assert_allclose(sum64(dk), 0.0, atol=tol)
     np.testing.assert_allclose(sum64(dv), sum64(inp["do"]), atol=tol)
+
+
+@pytest.mark.slow
+def test_config_causal128k_fwd_bwd():
+    """The bench's workload (128K causal) at full size."""
+    _full_size_fwd_bwd("causal128k")
+
+
+@pytest.mark.slow
+def test_config_packed128k_fwd_bwd():
+    """128K packed documents (segment masking across documents) at full size, forward and backward."""
+    _full_size_fwd_bwd("packed128k")

@@ -172,8 +172,10 @@ def test_fully_masked_rows_give_zero_and_neg_inf():
 
 
 def test_step_finalize_merge_follow_the_ring():
-    """Drive ra_step over the ring by hand, then finalize / merge partials."""
-    for dtype in ("f32", "bf16"):
+    """Drive the fp32 ra_step over the ring by hand, then finalize / merge partials,
+    held to the fp32 bound 1e-5 (the bf16 tensor-core step is tested in
+    test_gpu_step.py under the bf16 rule)."""
+    for dtype in ("f32",):
         w, inp = make_small(64, 1024, 4, 1, "packed", "neginf", 1, 2, dtype=dtype)
         q, k, v, bias, seg = inp["q"], inp["k"], inp["v"], inp["bias"], inp["seg"]
         blk = w.S // w.P
@@ -193,8 +195,8 @@ def test_step_finalize_merge_follow_the_ring():
             lses.append(lse)
         o = torch.cat(outs, 1)
         lse = torch.cat(lses, 2)
-        assert compare(to64(o), ro, "f32", max_abs=2e-5).ok
-        assert_lse(to64(lse), rl, 2e-5)
+        assert compare(to64(o), ro, "f32").ok
+        assert_lse(to64(lse), rl, LSE_F32)
         # merge: partial over keys of the first half + partial over the second half
         half = w.S // 2
         parts = []
@@ -204,8 +206,8 @@ def test_step_finalize_merge_follow_the_ring():
                          seg_q=seg, seg_k=seg[:, lo:hi].contiguous(), causal_block_size=1)
             parts.append(ra.finalize(acc, m, l, torch.float32))
         mo, ml = ra.lse_merge(parts[0][0], parts[0][1], parts[1][0], parts[1][1])
-        assert compare(to64(mo), ro, "f32", max_abs=2e-5).ok
-        assert_lse(to64(ml), rl, 2e-5)
+        assert compare(to64(mo), ro, "f32").ok
+        assert_lse(to64(ml), rl, LSE_F32)
 
 
 # ---------------------------------------------------------------- full-size configs

@@ -38,34 +38,46 @@ def _call_static(inp, w, o, lse):
                                          torch.cuda.current_stream().cuda_stream)
 
 
-def test_static_scratch_forward_matches_workspace_forward_twice():
+CASES = [
+    # (workload, random bias with -inf keys)
+    (dict(B=2, H=2, D=128, S=1024, P=4, chunk=256, causal_block_size=1, segments="packed", doc_lo=40, doc_hi=300,
+          seed=31), True),
+    (dict(B=1, H=3, D=64, S=640, P=5, chunk=128, causal_block_size=None, segments="packed", doc_lo=50, doc_hi=200,
+          seed=32), True),
+    # neither bias nor segments: no scratch is needed and none is looked up
+    (dict(B=1, H=2, D=128, S=768, P=3, chunk=256, causal_block_size=1, seed=33), False),
+    # fp32 inputs (CUDA-core path) with segment metadata in the static array
+    (dict(B=1, H=2, D=64, S=512, P=2, chunk=256, causal_block_size=1, dtype="f32", segments="packed", doc_lo=40,
+          doc_hi=200, seed=34), False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=["bf16-D128-seg-bias", "bf16-D64-seg-bias", "bf16-plain", "f32-seg"])
+def test_static_scratch_forward_matches_workspace_forward_twice(case):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     dev = torch.device("cuda:0")
-    cases = [
-        W.small_workload(B=2, H=2, D=128, S=1024, P=4, chunk=256, causal_block_size=1, segments="packed",
-                         doc_lo=40, doc_hi=300, seed=31),
-        W.small_workload(B=1, H=3, D=64, S=640, P=5, chunk=128, causal_block_size=None, segments="packed",
-                         doc_lo=50, doc_hi=200, seed=32),
-    ]
-    for w in cases:
-        inp = W.make_inputs(w, dev)
+    spec, with_bias = case
+    w = W.small_workload(**spec)
+    inp = W.make_inputs(w, dev)
+    if with_bias:
         g = torch.Generator(device="cpu").manual_seed(w.seed)
         bias = torch.randn((w.B, w.S), generator=g)
         bias[:, torch.randint(0, w.S, (w.S // 7,), generator=g)] = float("-inf")
         inp["bias"] = bias.to(dev)
-        ref_o, ref_lse = ra.ringattention(inp["q"], inp["k"], inp["v"], inp["bias"], inp["seg"],
-                                          query_chunk_size=w.chunk, key_chunk_size=w.chunk,
-                                          causal_block_size=w.causal_block_size, ring_size=w.P)
-        for _ in range(2):                                   # two calls in a row share the static array
-            o = torch.full_like(inp["q"], float("nan"))
-            lse = torch.full((w.B, w.H, w.S), float("nan"), dtype=torch.float32, device=dev)
-            assert _call_static(inp, w, o, lse) == 0
-            torch.cuda.synchronize()
-            assert ra.device_status() == 0
-            res = compare(to64(o), to64(ref_o), "bf16")
-            assert res.ok, str(res)
-            assert torch.equal(o, ref_o) and torch.equal(lse, ref_lse)
+    ref_o, ref_lse = ra.ringattention(inp["q"], inp["k"], inp["v"], inp["bias"], inp["seg"],
+                                      query_chunk_size=w.chunk, key_chunk_size=w.chunk,
+                                      causal_block_size=w.causal_block_size, ring_size=w.P)
+    kind = "f32" if w.dtype == "f32" else "bf16"
+    for _ in range(2):                                   # two calls in a row share the static array
+        o = torch.full_like(inp["q"], float("nan"))
+        lse = torch.full((w.B, w.H, w.S), float("nan"), dtype=torch.float32, device=dev)
+        assert _call_static(inp, w, o, lse) == 0
+        torch.cuda.synchronize()
+        assert ra.device_status() == 0
+        res = compare(to64(o), to64(ref_o), kind)
+        assert res.ok, str(res)
+        assert torch.equal(o, ref_o) and torch.equal(lse, ref_lse)
 
 
 def test_static_scratch_rejects_oversized_problems():
