@@ -368,6 +368,75 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_ffn(args):
+    """--mode ffn: the blockwise feed-forward network (ra_feedforward, SwiGLU) over
+    the workload's tokens: T = B*S tokens of d_model = H*D, d_ff = 11008 (the
+    LLaMA-7B ratio for d_model 4096), chunk of 8192 tokens.  Algorithmic
+    work 6*T*d_model*d_ff flop (three products)."""
+    import torch
+
+    import long_context_exact_ordered_b200 as ra
+    import workloads as W
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    w = W.WORKLOADS[args.workload]
+    T, dm, dff, chunk = w.B * w.S, w.H * w.D, args.ffn_dff, args.ffn_chunk
+    g = torch.Generator(device=dev).manual_seed(w.seed + rank)
+    x = torch.randn((T, dm), generator=g, device=dev).to(torch.bfloat16)
+    w1 = (torch.randn((dff, dm), generator=g, device=dev) * dm ** -0.5).to(torch.bfloat16)
+    w3 = (torch.randn((dff, dm), generator=g, device=dev) * dm ** -0.5).to(torch.bfloat16)
+    w2 = (torch.randn((dm, dff), generator=g, device=dev) * dff ** -0.5).to(torch.bfloat16)
+    y = torch.empty_like(x)
+    ws = torch.empty(ra.load().ra_feedforward_workspace_size(chunk, dff), dtype=torch.uint8, device=dev)
+    step = lambda: ra.blockwise_feedforward(x, w1, w3, w2, chunk_size=chunk, out=y, workspace=ws)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    sampler = ClockSampler(f"GPU-{props.uuid}" if not str(props.uuid).startswith("GPU-") else str(props.uuid))
+    barrier(world)
+    torch.cuda.synchronize()
+    sampler.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    fl = 6.0 * T * dm * dff
+    value = aggregate(fl * args.steps, ms / 1e3, world) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    n_chunks = (T + chunk - 1) // chunk
+    out = {
+        "metric": "blockwise feed-forward TFLOP/s", "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": f"ffn_{w.name}", "tokens": T, "d_model": dm, "d_ff": dff, "chunk": chunk,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "no flush: the weights (%.2f GB) and activations exceed the 126 MB L2" % (3 * dm * dff * 2 / 1e9)},
+        "mode": "blockwise feed-forward (SwiGLU)", "clocks": clocks, "e2e": None,
+        "gpu_launches": 2 * n_chunks * args.steps,
+        "roofline": {"bound": "tensor", "kernel": "ra_ffn_gemm_kernel", "achieved": round(value / world, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(value / world / peak, 4),
+                     "frac_of_burst_peak": round(value / world / burst, 4),
+                     "peak_source": f"{peak_src} bf16_tflops_sustained", "traffic": None},
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
 def run_ring(args):
     """--ring: the forward with the sequence sharded over the N ranks, key/value
     blocks exchanged round the ring over NCCL (long_context_exact_ordered_b200.ring,
@@ -593,9 +662,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="causal128k")
-    ap.add_argument("--mode", choices=["fwdbwd", "fwd", "step"], default="fwdbwd",
+    ap.add_argument("--ffn-dff", type=int, default=11008, help="--mode ffn: hidden width d_ff")
+    ap.add_argument("--ffn-chunk", type=int, default=8192, help="--mode ffn: tokens per chunk")
+    ap.add_argument("--mode", choices=["fwdbwd", "fwd", "step", "ffn"], default="fwdbwd",
                     help="fwdbwd: one step = forward + backward (default); fwd: forward only; step: the forward "
-                         "as P*P per-step calls (ra_step, tensor cores) plus ra_finalize per rank")
+                         "as P*P per-step calls (ra_step, tensor cores) plus ra_finalize per rank; ffn: the "
+                         "blockwise feed-forward network over the workload's tokens")
     ap.add_argument("--ring", action="store_true",
                     help="forward with the sequence sharded over the N ranks (ring of NCCL exchanges) instead of "
                          "N independent replicas")
@@ -613,6 +685,8 @@ def main(argv=None):
         run_reference(args)
     elif args.ring:
         run_ring(args)
+    elif args.mode == "ffn":
+        run_ffn(args)
     else:
         run_ours(args)
 

@@ -188,6 +188,26 @@ int ra_finalize(const ra_tensor* o_acc, const ra_tensor* m, const ra_tensor* l, 
 int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* o_b, const ra_tensor* lse_b,
                  ra_tensor* o_out, ra_tensor* lse_out, void* stream);
 
+/* Blockwise feed-forward network, exported next to ringattention
+ * ("RingAttention核心功能全解析" 核心API调用: from ringattention import
+ * ringattention, blockwise_feedforward).  The page prints no formula; the
+ * reading taken is the position-wise feed-forward network of the LLaMA
+ * configuration the page shards, a SwiGLU without biases:
+ *   h_t = silu(x_t W1^T) * (x_t W3^T),  y_t = h_t W2^T,  silu(a) = a / (1 + e^-a),
+ * evaluated chunk_size tokens at a time, so only one chunk's h [chunk, d_ff]
+ * (bf16, in `workspace`) is ever held: memory linear in the sequence length.
+ * Both products run on the tensor cores (bf16 in, fp32 accumulate); h is
+ * rounded to bf16 between them, y to bf16 at the end.
+ *  x: bf16 [T, d_model]; w1, w3: bf16 [d_ff, d_model]; w2: bf16 [d_model, d_ff]
+ *  (weights output-major, like a linear layer's); y: bf16 [T, d_model].  Rows
+ *  contiguous (stride[1] = 1), 16-byte aligned bases and row strides;
+ *  d_model and d_ff multiples of 32.
+ *  workspace: device, at least ra_feedforward_workspace_size(chunk_size, d_ff)
+ *  bytes, 256-byte aligned. */
+size_t ra_feedforward_workspace_size(int64_t chunk_size, int64_t d_ff);
+int ra_feedforward(const ra_tensor* x, const ra_tensor* w1, const ra_tensor* w3, const ra_tensor* w2, ra_tensor* y,
+                   int64_t chunk_size, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Forward that allocates nothing, for callers that cannot allocate device
  * memory: a host program that links only this library and owns no device
  * allocator, or code running under a fixed, pre-planned memory budget where a

@@ -7,6 +7,7 @@ ABI, include/ringattn.h); this package only marshals torch tensors into it.
 from .api import (  # noqa: F401
     HostStep,
     RingAttentionFunction,
+    blockwise_feedforward,
     count_visible_pairs,
     device_status,
     finalize,
@@ -26,5 +27,5 @@ from ._lib import RingAttnError, load  # noqa: F401
 __all__ = [
     "ringattention", "ringattention_backward", "ringattention_static", "ring_step", "init_state", "finalize", "lse_merge",
     "device_status", "selftest_timeout", "count_visible_pairs", "ring_schedule", "workspace_size", "RingAttentionFunction", "visible_count_probe",
-    "HostStep", "RingAttnError", "load",
+    "HostStep", "RingAttnError", "load", "blockwise_feedforward",
 ]

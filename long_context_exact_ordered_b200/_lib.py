@@ -66,6 +66,8 @@ SIGNATURES = {
     "ra_lse_merge": (ctypes.c_int, [_T, _T, _T, _T, _T, _T, _vp]),
     "ra_train_step_host": (ctypes.c_int, [ctypes.POINTER(RaHostStep), _T, _T, _P, ctypes.c_int64, _vp,
                                           ctypes.c_size_t, _vp, _vp, _vp]),
+    "ra_feedforward_workspace_size": (ctypes.c_size_t, [ctypes.c_int64, ctypes.c_int64]),
+    "ra_feedforward": (ctypes.c_int, [_T, _T, _T, _T, _T, ctypes.c_int64, _vp, ctypes.c_size_t, _vp]),
     "ra_get_device_status": (ctypes.c_int, [_vp]),
     "ra_selftest_timeout": (ctypes.c_int, [ctypes.c_int64, _vp]),
     "ra_strerror": (ctypes.c_char_p, [ctypes.c_int]),

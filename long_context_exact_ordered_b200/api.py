@@ -217,6 +217,26 @@ def lse_merge(o_a, lse_a, o_b, lse_b, out=None, lse_out=None):
     return out, lse_out
 
 
+def blockwise_feedforward(x, w1, w3, w2, chunk_size=4096, out=None, workspace=None):
+    """SwiGLU feed-forward y = (silu(x W1^T) * (x W3^T)) W2^T, chunk_size tokens
+    at a time (see ra_feedforward).  x: bf16 [T, d_model] (a [..., d_model]
+    tensor is flattened); w1, w3: [d_ff, d_model]; w2: [d_model, d_ff]."""
+    shape = x.shape
+    x2 = x.reshape(-1, shape[-1])
+    T, dff = x2.shape[0], w1.shape[0]
+    y = torch.empty_like(x2) if out is None else out.reshape(-1, shape[-1])
+    lib = load()
+    chunk = max(1, min(int(chunk_size), max(T, 1)))
+    need = lib.ra_feedforward_workspace_size(chunk, dff)
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, x.device)
+    ts = [_tensor(t) for t in (x2, w1, w3, w2, y)]
+    code = lib.ra_feedforward(*[ctypes.byref(t) for t in ts], chunk, None if workspace is None else workspace.data_ptr(),
+                              need, _stream())
+    check(code, "ra_feedforward")
+    return y.reshape(shape)
+
+
 def device_status(stream=None) -> int:
     """Synchronize and return (then clear) the device-side status word."""
     s = _stream() if stream is None else stream

@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <nvtx3/nvToolsExt.h>   // header-only; a no-op unless a profiler injects itself
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -16,6 +17,7 @@
 #include "ra_common.cuh"
 #include "ra_fwd_sm100.cuh"
 #include "ra_bwd_sm100.cuh"
+#include "ra_ffn_sm100.cuh"
 #include "ra_simt.cuh"
 
 using namespace ra;
@@ -227,7 +229,36 @@ int make_tmap_bshd(CUtensorMap* m, const ra_tensor* t, int rows) {
   return cu_fail(r, "cuTensorMapEncodeTiled (bf16 [B,S,H,D])");
 }
 
+// bf16 row-major matrix [rows, cols] (row stride in elements) -> 2-D map
+// (cols, rows), box 64 x box_rows, 128-byte swizzle.
+int make_tmap_rows(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t row_stride, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cu_fail(CUDA_ERROR_NOT_FOUND, "cuTensorMapEncodeTiled entry point");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return cu_fail(r, "cuTensorMapEncodeTiled (bf16 matrix)");
+}
+
 int last_cuda(const char* what = "kernel launch") { return cuda_fail(cudaGetLastError(), what); }
+
+// fp32 [BH][S][D] workspace -> 3-D map (D, S, BH), box D x rows x 1, no swizzle.
+int make_tmap_dqacc(CUtensorMap* m, float* base, int64_t BH, int64_t S, int64_t D, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return cu_fail(CUDA_ERROR_NOT_FOUND, "cuTensorMapEncodeTiled entry point");
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)S * D * 4};
+  cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return cu_fail(r, "cuTensorMapEncodeTiled (fp32 dQ accumulator)");
+}
 
 // NVTX range around one entry point's host work (its launches show under it
 // in an nsys / ncu timeline).
@@ -423,7 +454,7 @@ struct FwdSimtLaunch {
 template <int D>
 struct BwdSm100Launch {
   using L = BwdLayout<D>;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   BwdParams prm;
   int64_t grid = 0;
 
@@ -433,6 +464,8 @@ struct BwdSm100Launch {
     RA_TRY(make_tmap_bshd(&tk, k, kTile));
     RA_TRY(make_tmap_bshd(&tv, v, kTile));
     RA_TRY(make_tmap_bshd(&tdo, d_o, L::QT));
+    RA_TRY(make_tmap_dqacc(&tdq, reinterpret_cast<float*>(ws + w.dqacc), q->shape[0] * q->shape[2], q->shape[1],
+                           L::D, L::QT));
     std::memset(&prm, 0, sizeof(prm));
     prm.rd = rd;
     prm.B = (int32_t)q->shape[0];
@@ -464,18 +497,12 @@ struct BwdSm100Launch {
 #endif
     grid = (int64_t)rd.ntiles * prm.B * prm.H;
     if (grid > INT32_MAX) return RA_ERR_UNSUPPORTED;
-    RA_TRY(cuda_fail(
+    return cuda_fail(
         cudaFuncSetAttribute(ra_bwd_sm100_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_ALLOC),
-        "cudaFuncSetAttribute (backward kernel)"));
-    // The register split must fit in what the block is launched with.
-    cudaFuncAttributes fa;
-    RA_TRY(cuda_fail(cudaFuncGetAttributes(&fa, ra_bwd_sm100_kernel<D>), "cudaFuncGetAttributes (backward kernel)"));
-    if (128 * (L::REGS_WG0 + 2 * L::REGS_SOFTMAX + L::REGS_READOUT) > L::THREADS * fa.numRegs)
-      return RA_ERR_UNSUPPORTED;
-    return RA_OK;
+        "cudaFuncSetAttribute (backward kernel)");
   }
   int launch(cudaStream_t st) const {
-    ra_bwd_sm100_kernel<D><<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, prm);
+    ra_bwd_sm100_kernel<D><<<(unsigned)grid, L::THREADS, L::SMEM_ALLOC, st>>>(tq, tk, tv, tdo, tdq, prm);
     return last_cuda();
   }
 };
@@ -862,6 +889,92 @@ int ra_lse_merge(const ra_tensor* o_a, const ra_tensor* lse_a, const ra_tensor* 
   if (bind_device(o_a->data) < 0) return RA_ERR_CUDA;
   lse_merge_kernel<<<(unsigned)ceil_div64(n, 128), 128, 0, static_cast<cudaStream_t>(stream)>>>(a);
   return last_cuda();
+}
+
+size_t ra_feedforward_workspace_size(int64_t chunk_size, int64_t d_ff) {
+  if (chunk_size < 1 || d_ff < 1) return (size_t)-1;
+  return align256((size_t)chunk_size * (size_t)d_ff * 2);
+}
+
+int ra_feedforward(const ra_tensor* x, const ra_tensor* w1, const ra_tensor* w3, const ra_tensor* w2, ra_tensor* y,
+                   int64_t chunk_size, void* workspace, size_t workspace_bytes, void* stream) {
+  const NvtxRange nvtx_range("ra_feedforward");
+  if (!x || !w1 || !w3 || !w2 || !y) return RA_ERR_NULL;
+  for (const ra_tensor* t : {x, w1, w3, w2, (const ra_tensor*)y}) {
+    if (t->ndim != 2) return RA_ERR_SHAPE;
+    if (t->dtype != RA_BF16) return RA_ERR_DTYPE;
+  }
+  const int64_t T = x->shape[0], dm = x->shape[1], dff = w1->shape[0];
+  if (T < 0 || dm < 1 || dff < 1) return RA_ERR_SHAPE;
+  if (w1->shape[1] != dm || w3->shape[0] != dff || w3->shape[1] != dm || w2->shape[0] != dm || w2->shape[1] != dff ||
+      y->shape[0] != T || y->shape[1] != dm)
+    return RA_ERR_SHAPE;
+  for (const ra_tensor* t : {x, w1, w3, w2, (const ra_tensor*)y}) {
+    if (t->stride[1] != 1) return RA_ERR_STRIDE;
+    if (reinterpret_cast<uintptr_t>(t->data) % 16 || (t->stride[0] * 2) % 16 || t->stride[0] < t->shape[1])
+      return RA_ERR_STRIDE;
+    if (!t->data && t->shape[0] * t->shape[1] > 0) return RA_ERR_NULL;
+  }
+  // output columns are written 32 at a time; rows of the reduction are read by TMA
+  if (dm % 32 || dff % 32) return RA_ERR_UNSUPPORTED;
+  if (chunk_size < 1) return RA_ERR_DIVISIBILITY;
+  if (T == 0) return RA_OK;
+  const int64_t chunk = chunk_size < T ? chunk_size : T;
+  if (chunk > INT32_MAX / 2 || T > INT32_MAX / 2 || dff > INT32_MAX / 2 || dm > INT32_MAX / 2) return RA_ERR_UNSUPPORTED;
+  const size_t need = ra_feedforward_workspace_size(chunk, dff);
+  if (!workspace || workspace_bytes < need || reinterpret_cast<uintptr_t>(workspace) % 256) return RA_ERR_WORKSPACE;
+  const int major = bind_device(x->data);
+  if (major < 0) return RA_ERR_CUDA;
+  if (major != 10) return RA_ERR_UNSUPPORTED;
+  int dev = 0, sms = 0;
+  RA_TRY(cuda_fail(cudaGetDevice(&dev), "cudaGetDevice"));
+  RA_TRY(cuda_fail(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev), "cudaDeviceGetAttribute"));
+  // set-up first: every tensor map and attribute, then the launches
+  __nv_bfloat16* hbuf = static_cast<__nv_bfloat16*>(workspace);
+  CUtensorMap tx, tw1, tw3, tw2, th;
+  RA_TRY(make_tmap_rows(&tx, x->data, T, dm, x->stride[0], FfnLayout::BM));
+  RA_TRY(make_tmap_rows(&tw1, w1->data, dff, dm, w1->stride[0], 128));
+  RA_TRY(make_tmap_rows(&tw3, w3->data, dff, dm, w3->stride[0], 128));
+  RA_TRY(make_tmap_rows(&tw2, w2->data, dm, dff, w2->stride[0], FfnLayout::BN));
+  RA_TRY(make_tmap_rows(&th, hbuf, chunk, dff, dff, FfnLayout::BM));
+  RA_TRY(cuda_fail(cudaFuncSetAttribute(ra_ffn_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        FfnLayout::SMEM_ALLOC),
+                   "cudaFuncSetAttribute (feed-forward gated GEMM)"));
+  RA_TRY(cuda_fail(cudaFuncSetAttribute(ra_ffn_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        FfnLayout::SMEM_ALLOC),
+                   "cudaFuncSetAttribute (feed-forward GEMM)"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(y->data);
+  for (int64_t m0 = 0; m0 < T; m0 += chunk) {
+    const int64_t M = T - m0 < chunk ? T - m0 : chunk;
+    FfnParams g{};
+    g.M = (int32_t)M;
+    g.a_row0 = (int32_t)m0;
+    g.c_row0 = 0;
+    g.N = (int32_t)dff;
+    g.K = (int32_t)dm;
+    g.n_tiles = (int32_t)((dff + 127) / 128);
+    g.m_tiles = (int32_t)((M + FfnLayout::BM - 1) / FfnLayout::BM);
+    g.c = hbuf;
+    g.ldc = dff;
+    const int grid1 = (int)std::min<int64_t>((int64_t)g.n_tiles * g.m_tiles, sms);
+    ra_ffn_gemm_kernel<true><<<grid1, FfnLayout::THREADS, FfnLayout::SMEM_ALLOC, st>>>(tx, tw1, tw3, g);
+    RA_TRY(last_cuda("feed-forward gated GEMM launch"));
+    FfnParams o{};
+    o.M = (int32_t)M;
+    o.a_row0 = 0;
+    o.c_row0 = m0;
+    o.N = (int32_t)dm;
+    o.K = (int32_t)dff;
+    o.n_tiles = (int32_t)((dm + FfnLayout::BN - 1) / FfnLayout::BN);
+    o.m_tiles = g.m_tiles;
+    o.c = yp;
+    o.ldc = y->stride[0];
+    const int grid2 = (int)std::min<int64_t>((int64_t)o.n_tiles * o.m_tiles, sms);
+    ra_ffn_gemm_kernel<false><<<grid2, FfnLayout::THREADS, FfnLayout::SMEM_ALLOC, st>>>(th, tw2, tw2, o);
+    RA_TRY(last_cuda("feed-forward GEMM launch"));
+  }
+  return RA_OK;
 }
 
 int ra_forward_static(const ra_tensor* q, const ra_tensor* k, const ra_tensor* v, const ra_tensor* attention_bias,

@@ -4,51 +4,35 @@
 // "RingAttention核心功能全解析", 核心API调用).
 //
 // Work unit = one (batch, head, 128-key tile).  The key/value tile stays
-// resident while 128-row query tiles stream past in ring order: in the ring,
+// resident while 64-row query tiles stream past in ring order: in the ring,
 // a key/value block of ring block src meets query block (src + t) mod P at
 // step t (page "Ring Attention技术解析" §2.2), so dK and dV accumulate as the
 // block travels.  Per query tile i (all products on the tensor cores, fp32
-// accumulators in TMEM, M = N = 128 everywhere):
-//   S^T  = K Q_i^T              (SS, K-major)                 -> TMEM [128 x 128]
-//   dP^T = V dO_i^T             (SS, K-major)                 -> TMEM [128 x 128]
+// accumulators in TMEM, M = 128 everywhere):
+//   S^T  = K Q_i^T              (SS, K-major)            -> TMEM [128 x 64]
+//   dP^T = V dO_i^T             (SS, K-major)            -> TMEM [128 x 64]
 //   P^T  = exp2(S^T log2e/sqrt(D) - lse_i log2e) (masked), dS^T = P^T (dP^T - Delta_i)
 //   dV  += P^T dO_i             (TS: P^T bf16 in TMEM, dO MN-major)
 //   dK  += dS^T Q_i             (TS: dS^T bf16 in TMEM, Q MN-major)
-//   dQ^T = K^T dS^T             (SS: K and dS^T both MN-major) -> TMEM [128 x 128]
-// dQ^T is read back by a dedicated warpgroup and added straight from
-// registers into the fp32 dQ workspace with coalesced global reductions (dQ
-// gathers contributions from every key tile); shared memory, whose
-// bandwidth the tensor cores' operand reads mostly use, is not involved.
-//
-// Why 128 x 128: every product then has N = 128, where a shared-memory
-// operand read (A 4 KB + B 4 KB per K-step) keeps pace with the tensor core
-// (64 cycles each); with 64-query tiles the three SS products ran at N = 64
-// and were bound by shared-memory bandwidth, and the stationary K and V were
-// re-read twice as often per query.
+//   dQ^T = K^T dS^T             (SS: K and dS^T both MN-major) -> TMEM [128 x 64]
+// dQ^T is read back by a dedicated warpgroup, staged in shared memory as a
+// [64 queries x D] fp32 tile and added into the fp32 dQ workspace with one
+// TMA bulk reduce-add per tile (dQ gathers contributions from every key tile).
 //
 // Roles (512 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer,
-// warps 4-7 and 12-15 "softmax" (thread = key row; warpgroup w takes query
-// columns [64w, 64w + 64) of each tile, in two chunks of 32: P^T, dS^T, then
-// dK (w = 0) or dV (w = 1) in the epilogue), warps 8-11 dQ readout (thread =
-// head-dim lane d of dQ^T).  setmaxnreg moves registers from warpgroup 0 and
-// the readout group to the two softmax groups.
+// warps 4-7 and 12-15 "softmax" (thread = key row; the two warpgroups take
+// query columns 0-31 and 32-63 of each tile: P^T, dS^T, then dK resp. dV in
+// the epilogue), warps 8-11 dQ readout (thread = head-dim lane d of dQ^T).
+// TMEM (512 columns): two 128-column slots, then dK [256,256+D), dV [256+D,256+2D).
+// Query tile n uses slot n % 2: S^T -> [0,64), dP^T -> [64,128); the softmax
+// group overwrites [0,32) with P^T and [32,64) with dS^T (bf16), and dQ^T(n)
+// lands in [64,128) once dP^T has been read.  A slot is reused two tiles
+// later, after the readout group has taken dQ^T out of it.
 //
-// TMEM (512 columns), a single slot:
-//   [0, 128)    S^T; query chunk c (queries 32c .. 32c+31) is overwritten by
-//               its own P^T (bf16 pairs) in [32c, 32c+16) and dS^T in
-//               [32c+16, 32c+32): each softmax thread writes only the
-//               columns of its own row it has already read;
-//   [128, 256)  dP^T, then dQ^T once the softmax has read dP^T;
-//   [256, 256+D) dK, [256+D, 256+2D) dV, accumulated over all query tiles.
-// MMA issue order (tile n):  dV(n)  dK(n)  S^T(n+1)  dQ^T(n)  | dP^T(n+1).
-// The tensor pipe runs one thread's MMAs in issue order: S^T(n+1) overwrites
-// P^T / dS^T(n) only after dV / dK(n) read them; dP^T(n+1) waits for the
-// readout of dQ^T(n).  The softmax exponentials of tile n+1 (P^T, signalled
-// separately) overlap dQ^T(n), the readout and dP^T(n+1); its dS^T work
-// overlaps dV(n+1).  dS^T also goes to shared memory (one buffer: softmax
-// n+1 writes it only after dP^T(n+1), which follows dQ^T(n)) as the B
-// operand of dQ^T.  At D = 64, dQ^T keeps M = 128 by reading a zero block as
-// the upper half of K^T, so only its first 64 rows are read out.
+// Overlap: with two slots the "head" products of tile n+1 (S^T, dP^T) are
+// computed while the softmax groups work on tile n; the issue order is given
+// at the MMA issuer below.  At D = 64, dQ^T keeps M = 128 by reading a zero
+// block as the upper half of K^T, so only its first 64 rows are read out.
 #pragma once
 
 #include <cuda.h>
@@ -64,13 +48,14 @@ template <int D_>
 struct BwdLayout {
   static constexpr int D = D_;                    // 64 or 128
   static constexpr int KCH = D / 64;              // 128-byte swizzle chunks along D
-  static constexpr int QT = kQTileBwd;            // 128 query rows per tile
+  static constexpr int QT = kQTileBwd;            // 64 query rows per tile
   static constexpr int KV_BYTES = kTile * D * 2;  // 32 KB at D = 128
-  static constexpr int CHUNK = kTile * 128;       // 16 KB box: 128 rows x 128 B
-  static constexpr int Q_BYTES = QT * D * 2;      // 32 KB at D = 128
-  static constexpr int DS_HALF = kTile * 64 * 2;  // 16 KB: 128 keys x 64 queries bf16
-  static constexpr int DS_BYTES = 2 * DS_HALF;    // 128 keys x 128 queries
-  static constexpr int NS = 2;                    // query-side stages (the next tile loads while one computes)
+  static constexpr int KV_CHUNK = kTile * 128;    // 16 KB box: 128 rows x 128 B
+  static constexpr int Q_BYTES = QT * D * 2;      // 16 KB at D = 128
+  static constexpr int Q_CHUNK = QT * 128;        // 8 KB box: 64 rows x 128 B
+  static constexpr int DS_BYTES = kTile * QT * 2; // 16 KB: 128 keys x 64 queries bf16
+  static constexpr int NS = 3;                    // query-side stages (two tiles in flight + one loading)
+  static constexpr int NSLOT = 2;                 // TMEM slots
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_BYTES;
   static constexpr int OFF_Q = OFF_V + KV_BYTES;
@@ -78,34 +63,36 @@ struct BwdLayout {
   static constexpr int OFF_DS = OFF_DO + NS * Q_BYTES;
   // dQ^T = K^T dS^T is an M = 128 product along D.  At D = 64 its second
   // 64-row half of A reads this zero block, so rows 64..127 of dQ^T are 0.
-  static constexpr int OFF_ZERO = OFF_DS + DS_BYTES;
-  static constexpr int ZERO_BYTES = D == 64 ? CHUNK : 0;
-  static constexpr uint32_t LBO_DQ = D == 128 ? CHUNK : OFF_ZERO - OFF_K;   // distance between the D halves
-  static constexpr int OFF_BAR = OFF_ZERO + ZERO_BYTES;
+  static constexpr int OFF_ZERO = OFF_DS + NSLOT * DS_BYTES;
+  static constexpr int ZERO_BYTES = D == 64 ? KV_CHUNK : 0;
+  static constexpr uint32_t LBO_DQ = D == 128 ? KV_CHUNK : OFF_ZERO - OFF_K;   // distance between the D halves
+  static constexpr int OFF_LD = OFF_ZERO + ZERO_BYTES;       // per stage: lse2[64], delta[64]
+  static constexpr int LD_BYTES = 2 * QT * 4;
+  static constexpr int OFF_DQS = OFF_LD + NS * LD_BYTES;    // dQ staging [64][D] fp32
+  static constexpr int DQS_BYTES = QT * D * 4;               // 32 KB at D = 128
+  static constexpr int OFF_BAR = OFF_DQS + DQS_BYTES;
   static constexpr int B_KV = 0;
   static constexpr int B_QF = 1;                  // [NS] query stage loaded
   static constexpr int B_QE = B_QF + NS;          // [NS] query stage free
-  static constexpr int B_SFULL = B_QE + NS;       // S^T computed
-  static constexpr int B_DPFULL = B_SFULL + 1;    // dP^T computed
-  static constexpr int B_PREADY = B_DPFULL + 1;   // P^T written (8 arrivals: softmax warps)
-  static constexpr int B_DSREADY = B_PREADY + 1;  // dS^T written to TMEM and shared memory (8 arrivals)
-  static constexpr int B_DQFULL = B_DSREADY + 1;  // dQ^T computed
-  static constexpr int B_SLOTFREE = B_DQFULL + 1; // dQ^T read out (4 arrivals: readout warps)
-  static constexpr int B_FINAL = B_SLOTFREE + 1;
-  static constexpr int NBAR = B_FINAL + 1;
+  static constexpr int B_SFULL = B_QE + NS;       // [NSLOT] S^T computed
+  static constexpr int B_DPFULL = B_SFULL + NSLOT;   // [NSLOT] dP^T computed
+  static constexpr int B_DSREADY = B_DPFULL + NSLOT; // [NSLOT] P^T, dS^T written (8 arrivals: softmax warps)
+  static constexpr int B_DQFULL = B_DSREADY + NSLOT; // [NSLOT] dQ^T computed
+  static constexpr int B_SLOTFREE = B_DQFULL + NSLOT;  // [NSLOT] dQ^T read out (4 arrivals: readout warps)
+  static constexpr int B_FINAL = B_SLOTFREE + NSLOT;
+  static constexpr int B_DQSFULL = B_FINAL + 1;      // staging written (4 arrivals)
+  static constexpr int B_DQSFREE = B_DQSFULL + 1;    // staging read by the bulk reduce
+  static constexpr int NBAR = B_DQSFREE + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_S = 0, COL_DP = 128;
+  static constexpr uint32_t SLOT_COLS = 128;
+  static constexpr uint32_t SLOT_ST = 0, SLOT_DPT = 64, SLOT_PT = 0, SLOT_DST = 32, SLOT_DQT = 64;
   static constexpr uint32_t COL_DK = 256, COL_DV = 256 + D;
   static constexpr int THREADS = 512;
-  // Register split (setmaxnreg), per thread: warpgroup 0 (producer, issuer),
-  // the two softmax warpgroups and the readout warpgroup.  The host checks
-  // 128 * (REGS_WG0 + 2 * REGS_SOFTMAX + REGS_READOUT) <= 512 * (registers
-  // per thread at launch) before launching, so every increase can be met.
-  static constexpr int REGS_WG0 = 96, REGS_SOFTMAX = 160, REGS_READOUT = 96;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+  static_assert(OFF_DQS % 128 == 0, "bulk reduce source alignment");
   static_assert(OFF_ZERO % 1024 == 0 && LBO_DQ % 16 == 0 && (LBO_DQ >> 4) < (1u << 14), "dQ^T operand layout");
   static_assert(D == 64 || D == 128, "head dim");
 };
@@ -132,9 +119,28 @@ struct BwdParams {
   int32_t* dbg_count;        // RA_DEBUG_COUNT builds: visible queries per key, [B, H, S], pre-zeroed
 };
 
-// fp32 add into global memory without a return value (a reduction at L2).
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+// Tensor bulk reduce-add shared -> global (3-D tile, fp32 add), tracked by a bulk group.
+__device__ __forceinline__ void tma_reduce_add_3d(const void* tmap, uint32_t src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+          reinterpret_cast<uint64_t>(tmap)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+// 1-D bulk copy global -> shared (16-byte aligned, size multiple of 16).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -145,7 +151,7 @@ template <int D>
 __global__ void __launch_bounds__(512, 1)
     ra_bwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                        const __grid_constant__ BwdParams p) {
+                        const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ BwdParams p) {
   using L = BwdLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -169,13 +175,16 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     mbar_init(bar(L::B_KV), 1);
     for (int i = 0; i < L::NS; ++i) { mbar_init(bar(L::B_QF + i), 1); mbar_init(bar(L::B_QE + i), 1); }
-    mbar_init(bar(L::B_SFULL), 1);
-    mbar_init(bar(L::B_DPFULL), 1);
-    mbar_init(bar(L::B_PREADY), 8);      // one arrive per softmax warp
-    mbar_init(bar(L::B_DSREADY), 8);
-    mbar_init(bar(L::B_DQFULL), 1);
-    mbar_init(bar(L::B_SLOTFREE), 4);    // one arrive per readout warp
+    for (int i = 0; i < L::NSLOT; ++i) {
+      mbar_init(bar(L::B_SFULL + i), 1);
+      mbar_init(bar(L::B_DPFULL + i), 1);
+      mbar_init(bar(L::B_DSREADY + i), 8);     // one arrive per softmax warp
+      mbar_init(bar(L::B_DQFULL + i), 1);
+      mbar_init(bar(L::B_SLOTFREE + i), 4);    // one arrive per readout warp
+    }
     mbar_init(bar(L::B_FINAL), 1);
+    mbar_init(bar(L::B_DQSFULL), 4);
+    mbar_init(bar(L::B_DQSFREE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -199,140 +208,144 @@ __global__ void __launch_bounds__(512, 1)
   // A key tile whose every bias is -inf is invisible to all queries.
   const bool dead = use_bias && !(km.z & kMetaAnyFinite);
 
-  if (warp < 4) {
-  regs_dec<L::REGS_WG0>();
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     // The whole warp runs the loop (its lanes scan 32 query tiles per
     // metadata round trip, q_iter_next_warp); one elected lane issues copies.
-    if (elect_one()) {
-      prefetch_tmap(&tm_q);
-      prefetch_tmap(&tm_k);
-      prefetch_tmap(&tm_v);
-      prefetch_tmap(&tm_do);
-      mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::KV_BYTES);
-      for (int c = 0; c < L::KCH; ++c) {
-        tma_load_4d(sbase + L::OFF_K + c * L::CHUNK, &tm_k, bar(L::B_KV), c * 64, h, (int)k0, b);
-        tma_load_4d(sbase + L::OFF_V + c * L::CHUNK, &tm_v, bar(L::B_KV), c * 64, h, (int)k0, b);
-      }
-    }
-    __syncwarp();
-    int n = 0;
-    if (!dead) {
-      QIter it;
-      q_iter_init(it, p.rd, k0, meta_b, use_seg);
-      for (int32_t q = q_iter_next_warp(it, p.rd); q >= 0; q = q_iter_next_warp(it, p.rd), ++n) {
-        const int st = n % L::NS;
-        if (n >= L::NS && !ra_wait_warp(bar(L::B_QE + st), ((n / L::NS) & 1) ^ 1, abort_flag)) break;
-        const int q0 = q * L::QT;
-        if (elect_one()) {
-          mbar_arrive_expect_tx(bar(L::B_QF + st), 2 * L::Q_BYTES);
-          for (int c = 0; c < L::KCH; ++c) {
-            tma_load_4d(sbase + L::OFF_Q + st * L::Q_BYTES + c * L::CHUNK, &tm_q, bar(L::B_QF + st), c * 64, h, q0, b);
-            tma_load_4d(sbase + L::OFF_DO + st * L::Q_BYTES + c * L::CHUNK, &tm_do, bar(L::B_QF + st), c * 64, h, q0,
-                        b);
-          }
+    {
+      if (elect_one()) {
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        prefetch_tmap(&tm_do);
+        mbar_arrive_expect_tx(bar(L::B_KV), 2 * L::KV_BYTES);
+        for (int c = 0; c < L::KCH; ++c) {
+          tma_load_4d(sbase + L::OFF_K + c * L::KV_CHUNK, &tm_k, bar(L::B_KV), c * 64, h, (int)k0, b);
+          tma_load_4d(sbase + L::OFF_V + c * L::KV_CHUNK, &tm_v, bar(L::B_KV), c * 64, h, (int)k0, b);
         }
-        __syncwarp();
       }
+      __syncwarp();
+      int n = 0;
+      if (!dead) {
+        QIter it;
+        q_iter_init(it, p.rd, k0, meta_b, use_seg);
+        const float* lse_row = p.lse2 + (int64_t)bh * p.s_pad;
+        const float* dl_row = p.delta + (int64_t)bh * p.s_pad;
+        for (int32_t q = q_iter_next_warp(it, p.rd); q >= 0; q = q_iter_next_warp(it, p.rd), ++n) {
+          const int st = n % L::NS;
+          if (n >= L::NS && !ra_wait_warp(bar(L::B_QE + st), ((n / L::NS) & 1) ^ 1, abort_flag)) break;
+          const int q0 = q * L::QT;
+          if (elect_one()) {
+            mbar_arrive_expect_tx(bar(L::B_QF + st), 2 * L::Q_BYTES + L::LD_BYTES);
+            for (int c = 0; c < L::KCH; ++c) {
+              tma_load_4d(sbase + L::OFF_Q + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_q, bar(L::B_QF + st), c * 64, h,
+                          q0, b);
+              tma_load_4d(sbase + L::OFF_DO + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_do, bar(L::B_QF + st), c * 64,
+                          h, q0, b);
+            }
+            bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES, lse_row + q0, L::QT * 4, bar(L::B_QF + st));
+            bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES + L::QT * 4, dl_row + q0, L::QT * 4, bar(L::B_QF + st));
+          }
+          __syncwarp();
+        }
+      }
+      ra_wait_drain(bar(L::B_KV), 0);
+      for (int i = n - L::NS; i < n; ++i)
+        if (i >= 0) ra_wait_drain(bar(L::B_QF + i % L::NS), (i / L::NS) & 1);
     }
-    ra_wait_drain(bar(L::B_KV), 0);
-    for (int i = n - L::NS; i < n; ++i)
-      if (i >= 0) ra_wait_drain(bar(L::B_QF + i % L::NS), (i / L::NS) & 1);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // The whole warp runs the issuer; one elected lane issues (ptx.cuh).
-    constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, L::QT, false, false);
-    constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);
-    constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, L::QT, true, true);
-    const uint32_t ka = sbase + L::OFF_K, va = sbase + L::OFF_V;
-    // Descriptors are built once per operand tile; the K-step offsets are
-    // added to the start-address field (address >> 4, no carry: shared
-    // memory ends below 2^18 bytes), keeping the issue loop short.
-    const uint64_t ka_k = smem_desc_sw128(ka, 16, 1024), va_k = smem_desc_sw128(va, 16, 1024);
-    const uint64_t ka_mn = smem_desc_sw128(ka, L::LBO_DQ, 1024);
-    const uint64_t ds_mn = smem_desc_sw128(sbase + L::OFF_DS, L::DS_HALF, 1024);
-    auto issue_sd = [&](uint32_t d_tmem, uint64_t a_desc, uint32_t b_base) {   // S^T or dP^T
-      const uint64_t b_desc = smem_desc_sw128(b_base, 16, 1024);
+    {   // the whole warp runs the issuer; one elected lane issues (ptx.cuh)
+      constexpr uint32_t IDESC_SD = idesc_bf16_f32(128, L::QT, false, false);
+      constexpr uint32_t IDESC_KV = idesc_bf16_f32(128, D, false, true);
+      constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, L::QT, true, true);
+      const uint32_t ka = sbase + L::OFF_K, va = sbase + L::OFF_V;
+      // Descriptors are built once per operand tile; the K-step offsets are
+      // added to the start-address field (address >> 4, no carry: shared
+      // memory ends below 2^18 bytes), keeping the issue loop short.
+      const uint64_t ka_k = smem_desc_sw128(ka, 16, 1024), va_k = smem_desc_sw128(va, 16, 1024);
+      const uint64_t ka_mn = smem_desc_sw128(ka, L::LBO_DQ, 1024);
+      auto issue_sd = [&](uint32_t d_tmem, uint64_t a_desc, uint32_t b_base) {   // S^T or dP^T
+        const uint64_t b_desc = smem_desc_sw128(b_base, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t o = ((kk / 4) * L::CHUNK + (kk % 4) * 32) >> 4;
-        mma_ss_w(d_tmem, a_desc + o, b_desc + o, IDESC_SD, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oa = ((kk / 4) * L::KV_CHUNK + (kk % 4) * 32) >> 4;
+          const uint32_t ob = ((kk / 4) * L::Q_CHUNK + (kk % 4) * 32) >> 4;
+          mma_ss_w(d_tmem, a_desc + oa, b_desc + ob, IDESC_SD, kk > 0);
+        }
+      };
+      auto issue_kv = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_base, bool acc) {   // dV or dK
+        const uint64_t b_desc = smem_desc_sw128(b_base, L::Q_CHUNK, 1024);
+#pragma unroll
+        for (int kk = 0; kk < L::QT / 16; ++kk)
+          mma_ts_w(d_tmem, a_tmem + kk * 8, b_desc + kk * (2048 >> 4), IDESC_KV, (acc || kk > 0) ? 1u : 0u);
+      };
+      auto issue_dq = [&](uint32_t d_tmem, uint32_t ds_base) {
+        const uint64_t b_desc = smem_desc_sw128(ds_base, L::DS_BYTES, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          mma_ss_w(d_tmem, ka_mn + kk * (2048 >> 4), b_desc + kk * (2048 >> 4), IDESC_DQ, kk > 0);
+      };
+      // number of query tiles this key tile visits
+      int N = 0;
+      if (!dead) {
+        QIter it;
+        q_iter_init(it, p.rd, k0, meta_b, use_seg);
+        while (q_iter_next_warp(it, p.rd) >= 0) ++N;
       }
-    };
-    // dV += P^T dO or dK += dS^T Q over the tile's 128 queries: K-step kk
-    // covers queries 16kk .. 16kk+15, held (bf16 pairs) in columns
-    // 32 (kk/2) + 8 (kk%2) + a_off of the S^T region (a_off 0: P^T, 16: dS^T).
-    auto issue_kv = [&](uint32_t d_tmem, uint32_t a_off, uint32_t b_base, bool acc) {
-      const uint64_t b_desc = smem_desc_sw128(b_base, L::CHUNK, 1024);
-#pragma unroll
-      for (int kk = 0; kk < L::QT / 16; ++kk)
-        mma_ts_w(d_tmem, tmem + L::COL_S + 32 * (kk / 2) + 8 * (kk % 2) + a_off, b_desc + kk * (2048 >> 4), IDESC_KV,
-                 (acc || kk > 0) ? 1u : 0u);
-    };
-    auto issue_dq = [&]() {   // dQ^T = K^T dS^T over the 128 keys
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        mma_ss_w(tmem + L::COL_DP, ka_mn + kk * (2048 >> 4), ds_mn + kk * (2048 >> 4), IDESC_DQ, kk > 0);
-    };
-    // number of query tiles this key tile visits
-    int N = 0;
-    if (!dead) {
-      QIter it;
-      q_iter_init(it, p.rd, k0, meta_b, use_seg);
-      while (q_iter_next_warp(it, p.rd) >= 0) ++N;
-    }
-    bool ok = ra_wait_warp(bar(L::B_KV), 0, abort_flag);
-    if (ok && N > 0) {
-      ok = ra_wait_warp(bar(L::B_QF + 0), 0, abort_flag);
-      if (ok) {
+      // Issue order (two TMEM slots, tile n in slot n % 2):
+      //   S^T(0) dP^T(0) S^T(1) dP^T(1) | tail(0) S^T(2) dP^T(2) | tail(1) S^T(3) dP^T(3) | ...
+      // with tail(n) = dQ^T(n), then dV(n), dK(n).  The tensor pipe runs one
+      // thread's MMAs in issue order, so S^T(n+2) may follow tail(n) at once
+      // (it overwrites P^T / dS^T(n) only after dV / dK(n) have read them);
+      // dP^T(n+2) overwrites dQ^T(n) and waits for its readout, which runs
+      // while dV, dK(n) and S^T(n+2) execute.  The softmax of tile n+1 has
+      // tail(n), S^T(n+2) and dP^T(n+2) of tensor work to hide behind.
+      bool ok = ra_wait_warp(bar(L::B_KV), 0, abort_flag);
+      auto head_s = [&](int m) -> bool {
+        const int st = m % L::NS;
+        if (!ra_wait_warp(bar(L::B_QF + st), (m / L::NS) & 1, abort_flag)) return false;
         tc_fence_after();
-        issue_sd(tmem + L::COL_S, ka_k, sbase + L::OFF_Q);
-        mma_commit_w(bar(L::B_SFULL));
-        issue_sd(tmem + L::COL_DP, va_k, sbase + L::OFF_DO);
-        mma_commit_w(bar(L::B_DPFULL));
-      }
-    }
-    for (int n = 0; ok && n < N; ++n) {
-      const int st = n % L::NS;
-      const uint32_t ph = n & 1;
-      if (!(ok = ra_wait_warp(bar(L::B_PREADY), ph, abort_flag))) break;
-      tc_fence_after();
-      issue_kv(tmem + L::COL_DV, 0, sbase + L::OFF_DO + st * L::Q_BYTES, n > 0);
-      if (!(ok = ra_wait_warp(bar(L::B_DSREADY), ph, abort_flag))) break;
-      tc_fence_after();
-      issue_kv(tmem + L::COL_DK, 16, sbase + L::OFF_Q + st * L::Q_BYTES, n > 0);
-      mma_commit_w(bar(L::B_QE + st));
-      const bool more = n + 1 < N;
-      if (more) {
-        const int st1 = (n + 1) % L::NS;
-        if (!(ok = ra_wait_warp(bar(L::B_QF + st1), ((n + 1) / L::NS) & 1, abort_flag))) break;
-        issue_sd(tmem + L::COL_S, ka_k, sbase + L::OFF_Q + st1 * L::Q_BYTES);
-        mma_commit_w(bar(L::B_SFULL));
-      }
-      issue_dq();
-      mma_commit_w(bar(L::B_DQFULL));
-      if (more) {
-        if (!(ok = ra_wait_warp(bar(L::B_SLOTFREE), ph, abort_flag))) break;
+        issue_sd(tmem + (m & 1) * L::SLOT_COLS + L::SLOT_ST, ka_k, sbase + L::OFF_Q + st * L::Q_BYTES);
+        mma_commit_w(bar(L::B_SFULL + (m & 1)));
+        return true;
+      };
+      auto head_dp = [&](int m) -> bool {
+        const int s = m & 1, st = m % L::NS;
+        if (m >= L::NSLOT && !ra_wait_warp(bar(L::B_SLOTFREE + s), ((m >> 1) - 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        issue_sd(tmem + L::COL_DP, va_k, sbase + L::OFF_DO + ((n + 1) % L::NS) * L::Q_BYTES);
-        mma_commit_w(bar(L::B_DPFULL));
+        issue_sd(tmem + s * L::SLOT_COLS + L::SLOT_DPT, va_k, sbase + L::OFF_DO + st * L::Q_BYTES);
+        mma_commit_w(bar(L::B_DPFULL + s));
+        return true;
+      };
+      for (int m = 0; ok && m < N && m < L::NSLOT; ++m) ok = head_s(m) && head_dp(m);
+      for (int t = 0; ok && t < N; ++t) {
+        const int s = t & 1, st = t % L::NS;
+        if (!(ok = ra_wait_warp(bar(L::B_DSREADY + s), (t >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t slot = tmem + s * L::SLOT_COLS;
+        issue_dq(slot + L::SLOT_DQT, sbase + L::OFF_DS + s * L::DS_BYTES);
+        mma_commit_w(bar(L::B_DQFULL + s));
+        issue_kv(tmem + L::COL_DV, slot + L::SLOT_PT, sbase + L::OFF_DO + st * L::Q_BYTES, t > 0);
+        issue_kv(tmem + L::COL_DK, slot + L::SLOT_DST, sbase + L::OFF_Q + st * L::Q_BYTES, t > 0);
+        mma_commit_w(bar(L::B_QE + st));
+        if (t + L::NSLOT < N) ok = head_s(t + L::NSLOT) && head_dp(t + L::NSLOT);
       }
+      mma_commit_w(bar(L::B_FINAL));
+      ra_wait_drain(bar(L::B_FINAL), 0);
     }
-    mma_commit_w(bar(L::B_FINAL));
-    ra_wait_drain(bar(L::B_FINAL), 0);
     __syncwarp();
-  }
   } else if ((warp >= 4 && warp < 8) || warp >= 12) {
     // ------------------------------------------------------------ softmax groups: one key row per thread
-    regs_inc<L::REGS_SOFTMAX>();
-    const int wg = warp >= 12;                       // query columns [64 wg, 64 wg + 64) of each tile
+    const int half = warp >= 12;                     // query columns [32*half, 32*half + 32) of each tile
+    const int c0 = half * 32;
     const int sub = warp & 3;
     const int row = sub * 32 + lane;
     const int64_t j = k0 + row;                      // this thread's key
     const bool row_valid = j < S;
     const int64_t jc = row_valid ? j : S - 1;
-    const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
+    const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
+    const uint32_t trow = tmem + lane_off;
     const int my_seg = use_seg ? p.seg[b * p.seg_sb + jc * p.seg_ss] : 0;
     float brow = 0.f;                                // bias of this key, log2 units
     if (use_bias) brow = p.bias[b * p.bias_sb + jc * p.bias_ss] * kLog2e;
@@ -342,8 +355,6 @@ __global__ void __launch_bounds__(512, 1)
     // causal block of the tile's last key (no per-tile division).
     const int64_t k_last_blk = cbs > 0 ? ((k0 + kTile - 1) / cbs) * (int64_t)cbs : 0;
     const float sc = p.scale_log2;
-    const float* lse2_bh = p.lse2 + (int64_t)bh * p.s_pad;
-    const float* delta_bh = p.delta + (int64_t)bh * p.s_pad;
 #ifdef RA_DEBUG_COUNT
     int dbg_vis = 0;
 #endif
@@ -353,109 +364,88 @@ __global__ void __launch_bounds__(512, 1)
       QIter it;
       q_iter_init(it, p.rd, k0, meta_b, use_seg);
       for (int32_t q = q_iter_next_warp(it, p.rd); q >= 0; q = q_iter_next_warp(it, p.rd), ++n) {
-        const uint32_t ph = n & 1;
+        const int st = n % L::NS, s = n & 1;
+        const uint32_t slot = trow + s * L::SLOT_COLS;
         const int64_t q0 = (int64_t)q * L::QT;
-        // the query tile's metadata load is issued before the wait, so it lands meanwhile
-        const int4 qm = meta_b ? load_meta(meta_b + q) : make_int4(0, 0, 3, 0);
+        // the query tile's metadata load is issued before the waits, so it lands meanwhile
+        const int4 qm = meta_b ? load_meta(meta_b + q0 / kTile) : make_int4(0, 0, 3, 0);
+        if (!(ok = ra_wait_warp(bar(L::B_QF + st), (n / L::NS) & 1, abort_flag))) break;
+        if (!(ok = ra_wait_warp(bar(L::B_SFULL + s), (n >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        uint32_t sr[32];
+        tmem_ld32(slot + L::SLOT_ST + c0, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) reg_fence(sr[c]);
+        float* x = reinterpret_cast<float*>(sr);
+        const float* nl = reinterpret_cast<const float*>(gbase + L::OFF_LD + st * L::LD_BYTES) + c0;   // -lse*log2e
+        const float* nd = nl + L::QT;                                                                 // -Delta
+        // x = S * log2(e)/sqrt(D) + bias(key) - lse(query) * log2(e), two columns per instruction
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          float b0 = nl[c], b1 = nl[c + 1];
+          if (use_bias) fadd2(b0, b1, b0, b1, brow, brow);
+          ffma2(x[c], x[c + 1], x[c], x[c + 1], sc, sc, b0, b1);
+        }
+        // per-element mask on causal-diagonal / ragged / mixed-segment tiles
         const bool need_causal = cbs > 0 && q0 < k_last_blk;
         const bool need_ragged = (q0 + L::QT > S) || (k0 + kTile > S);
         const bool need_seg = use_seg && !(qm.x == qm.y && km.x == km.y && qm.x == km.x);
-        const bool need_mask = need_causal || need_ragged || need_seg || !row_valid;
-        if (!(ok = ra_wait_warp(bar(L::B_SFULL), ph, abort_flag))) break;
-        tc_fence_after();
-        // ---- P^T for the group's two chunks of 32 queries
-        float pr[2][32];
+        if (need_causal || need_ragged || need_seg || !row_valid) {
+          const int64_t cmin64 = i_first - (q0 + c0);              // visible iff c >= cmin
+          const int cmin = cmin64 < 0 ? 0 : (cmin64 > 32 ? 32 : (int)cmin64);
+          const int64_t cmax64 = S - (q0 + c0);                    // valid iff c < cmax
+          const int cmax = row_valid ? (cmax64 > 32 ? 32 : (cmax64 < 0 ? 0 : (int)cmax64)) : 0;
+          uint32_t vb = ~0u;
+          if (need_seg) {
+            const int32_t* sp = p.seg + b * p.seg_sb;
+            vb = 0;
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int c = 2 * wg + jj;                 // chunk: queries 32c .. 32c+31 of the tile
-          uint32_t sr[32];
-          tmem_ld32(trow + L::COL_S + 32 * c, sr);
-          tmem_ld_wait();
-          float* x = pr[jj];
-          const float4* nl4 = reinterpret_cast<const float4*>(lse2_bh + q0 + 32 * c);   // -lse*log2e, broadcast
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float4 nl = __ldg(nl4 + e / 4);
-            if (use_bias) {
-              nl.x += brow; nl.y += brow; nl.z += brow; nl.w += brow;
-            }
-            reg_fence(sr[e]); reg_fence(sr[e + 1]); reg_fence(sr[e + 2]); reg_fence(sr[e + 3]);
-            ffma2(x[e], x[e + 1], __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), sc, sc, nl.x, nl.y);
-            ffma2(x[e + 2], x[e + 3], __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]), sc, sc, nl.z, nl.w);
-          }
-          if (need_mask) {
-            const int64_t qc0 = q0 + 32 * c;
-            const int64_t cmin64 = i_first - qc0;                  // visible iff e >= cmin
-            const int cmin = cmin64 < 0 ? 0 : (cmin64 > 32 ? 32 : (int)cmin64);
-            const int64_t cmax64 = S - qc0;                        // valid iff e < cmax
-            const int cmax = row_valid ? (cmax64 > 32 ? 32 : (cmax64 < 0 ? 0 : (int)cmax64)) : 0;
-            uint32_t vb = ~0u;
-            if (need_seg) {
-              const int32_t* sp = p.seg + b * p.seg_sb;
-              vb = 0;
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const int64_t i = qc0 + e < S ? qc0 + e : S - 1;
-                vb |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << e;
-              }
-            }
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const bool vis = e >= cmin && e < cmax && ((vb >> e) & 1u);
-              x[e] = vis ? x[e] : -INFINITY;
+            for (int c = 0; c < 32; ++c) {
+              const int64_t i = q0 + c0 + c < S ? q0 + c0 + c : S - 1;
+              vb |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << c;
             }
           }
-#ifdef RA_DEBUG_COUNT
-          // visible pairs as decided by this kernel's own tile skipping and masking
 #pragma unroll
-          for (int e = 0; e < 32; ++e) dbg_vis += x[e] != -INFINITY;
-#endif
-          uint32_t pp[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            x[e] = ex2_approx(x[e]);
-            x[e + 1] = ex2_approx(x[e + 1]);
-            pp[e >> 1] = pack_bf16x2(x[e], x[e + 1]);
+          for (int c = 0; c < 32; ++c) {
+            const bool vis = c >= cmin && c < cmax && ((vb >> c) & 1u);
+            x[c] = vis ? x[c] : -INFINITY;
           }
-          tmem_st16(trow + L::COL_S + 32 * c, pp);    // over this row's own, already read, S^T columns
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_PREADY));
-        // ---- dS^T = P^T (dP^T - Delta) for the same chunks
-        if (!(ok = ra_wait_warp(bar(L::B_DPFULL), ph, abort_flag))) break;
+#ifdef RA_DEBUG_COUNT
+        // visible pairs as decided by this kernel's own tile skipping and masking
+#pragma unroll
+        for (int c = 0; c < 32; ++c) dbg_vis += x[c] != -INFINITY;
+#endif
+        float pr[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pr[c] = ex2_approx(x[c]);
+        if (!(ok = ra_wait_warp(bar(L::B_DPFULL + s), (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
+        uint32_t dr[32];
+        tmem_ld32(slot + L::SLOT_DPT + c0, dr);
+        tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
-          const int c = 2 * wg + jj;
-          uint32_t dr[32];
-          tmem_ld32(trow + L::COL_DP + 32 * c, dr);
-          tmem_ld_wait();
-          const float4* nd4 = reinterpret_cast<const float4*>(delta_bh + q0 + 32 * c);   // -Delta, broadcast
-          uint32_t dd[16];
+        for (int c = 0; c < 32; ++c) reg_fence(dr[c]);
+        uint32_t pp[16], dd[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 nd = __ldg(nd4 + e / 4);
-            reg_fence(dr[e]); reg_fence(dr[e + 1]); reg_fence(dr[e + 2]); reg_fence(dr[e + 3]);
-            float t0, t1, t2, t3, s0, s1, s2, s3;
-            fadd2(t0, t1, __uint_as_float(dr[e]), __uint_as_float(dr[e + 1]), nd.x, nd.y);
-            fadd2(t2, t3, __uint_as_float(dr[e + 2]), __uint_as_float(dr[e + 3]), nd.z, nd.w);
-            fmul2(s0, s1, pr[jj][e], pr[jj][e + 1], t0, t1);
-            fmul2(s2, s3, pr[jj][e + 2], pr[jj][e + 3], t2, t3);
-            dd[e >> 1] = pack_bf16x2(s0, s1);
-            dd[(e >> 1) + 1] = pack_bf16x2(s2, s3);
-          }
-          tmem_st16(trow + L::COL_S + 32 * c + 16, dd);
-          // dS^T into shared memory for dQ^T = K^T dS^T (MN-major, 128-byte
-          // swizzle): queries 64h .. 64h+63 form half h; key row `row` is one
-          // 128-byte line of it, and 16-byte chunk u lands at u ^ (row % 8).
-          const uint32_t line = sbase + L::OFF_DS + (c / 2) * L::DS_HALF + row * 128;
+        for (int c = 0; c < 32; c += 2) {
+          float t0, t1, ds0, ds1;
+          fadd2(t0, t1, __uint_as_float(dr[c]), __uint_as_float(dr[c + 1]), nd[c], nd[c + 1]);   // dP - Delta
+          fmul2(ds0, ds1, pr[c], pr[c + 1], t0, t1);
+          pp[c >> 1] = pack_bf16x2(pr[c], pr[c + 1]);
+          dd[c >> 1] = pack_bf16x2(ds0, ds1);
+        }
+        // P^T and dS^T (bf16, two per column) into this slot's first half.
+        tmem_st16(slot + L::SLOT_PT + c0 / 2, pp);
+        tmem_st16(slot + L::SLOT_DST + c0 / 2, dd);
+        // dS^T into shared memory for dQ^T = K^T dS^T (MN-major, 128-byte swizzle):
+        // key row `row` is one 128-byte line; 16-byte chunk c lands at c ^ (row % 8).
+        const uint32_t line = sbase + L::OFF_DS + s * L::DS_BYTES + row * 128;
 #pragma unroll
-          for (int u4 = 0; u4 < 4; ++u4) {
-            const int u = (c % 2) * 4 + u4;
-            st_shared_v4(line + ((u ^ (row & 7)) << 4), dd[4 * u4], dd[4 * u4 + 1], dd[4 * u4 + 2], dd[4 * u4 + 3]);
-          }
+        for (int c = 0; c < 4; ++c) {
+          const int chunk = half * 4 + c;
+          st_shared_v4(line + ((chunk ^ (row & 7)) << 4), dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
         }
         fence_proxy_async_smem();
         tmem_st_wait();
@@ -463,25 +453,26 @@ __global__ void __launch_bounds__(512, 1)
         // one arrive per warp: per-lane arrives on one barrier serialise in the
         // shared-memory pipe, which the tensor cores' operand reads also use
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(L::B_DSREADY));
+        if (lane == 0) mbar_arrive(bar(L::B_DSREADY + s));
       }
     }
 #ifdef RA_DEBUG_COUNT
-    // the two query halves of a key row add their counts
+    // the two column halves of a key row add their counts
     if (row_valid && ok && p.dbg_count) atomicAdd(p.dbg_count + ((int64_t)b * p.H + h) * S + j, dbg_vis);
 #endif
-    // ---------------------------------------------------------- epilogue: dK (group 0) or dV (group 1)
+    // ---------------------------------------------------------- epilogue: dK (columns group 0) or dV (group 1)
     bool have = n > 0 && ok;
     if (have) have = ra_wait(bar(L::B_FINAL), 0, abort_flag);
     have = __all_sync(0xffffffffu, have);
     n = __shfl_sync(0xffffffffu, n, 0);
     tc_fence_after();
     {
-      const uint32_t col = wg == 0 ? L::COL_DK : L::COL_DV;
-      const float mul = wg == 0 ? p.scale : 1.f;
-      char* base = static_cast<char*>(wg == 0 ? p.dk : p.dv);
-      const int64_t sb = wg == 0 ? p.dk_sb : p.dv_sb, ss = wg == 0 ? p.dk_ss : p.dv_ss,
-                    sh = wg == 0 ? p.dk_sh : p.dv_sh;
+      const int which = half;
+      const uint32_t col = which == 0 ? L::COL_DK : L::COL_DV;
+      const float mul = which == 0 ? p.scale : 1.f;
+      char* base = static_cast<char*>(which == 0 ? p.dk : p.dv);
+      const int64_t sb = which == 0 ? p.dk_sb : p.dv_sb, ss = which == 0 ? p.dk_ss : p.dv_ss,
+                    sh = which == 0 ? p.dk_sh : p.dv_sh;
       const int64_t off = b * sb + jc * ss + h * sh;
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
@@ -516,48 +507,59 @@ __global__ void __launch_bounds__(512, 1)
         }
       }
     }
-  } else {
+  } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------ dQ readout: thread = head-dim lane d
-    // Each thread takes its row d of dQ^T (128 queries, in two halves) out of
-    // TMEM and adds the values straight into the fp32 accumulator
-    // dqacc[bh][q][d]: a warp's 32 lanes cover 32 consecutive d of one query
-    // row, so every reduction is one coalesced 128-byte request.  The slot
-    // is released as soon as the second half is in registers.
-    regs_dec<L::REGS_READOUT>();
     const int sub = warp & 3;
     const int d = sub * 32 + lane;
+    const bool leader = threadIdx.x == 256;
     const uint32_t trow = tmem + ((uint32_t)(sub * 32) << 16);
+    const uint32_t dqs = sbase + L::OFF_DQS;
+    bool pending = false;   // leader: a bulk reduce may still be reading the staging tile
     if (!dead) {
+      if (leader) prefetch_tmap(&tm_dq);
       QIter it;
       q_iter_init(it, p.rd, k0, meta_b, use_seg);
       int n = 0;
       for (int32_t q = q_iter_next_warp(it, p.rd); q >= 0; q = q_iter_next_warp(it, p.rd), ++n) {
-        if (!ra_wait_warp(bar(L::B_DQFULL), n & 1, abort_flag)) break;
+        const int s = n & 1;
+        if (!ra_wait_warp(bar(L::B_DQFULL + s), (n >> 1) & 1, abort_flag)) break;
         tc_fence_after();
-        const int64_t q0 = (int64_t)q * L::QT;
-        const int64_t rows = S - q0 < L::QT ? S - q0 : L::QT;   // the last query tile may be ragged
-        float* dst = p.dqacc + ((int64_t)bh * S + q0) * D + d;
+        uint32_t r[64];
+        tmem_ld32(trow + s * L::SLOT_COLS + L::SLOT_DQT, r);
+        tmem_ld32(trow + s * L::SLOT_COLS + L::SLOT_DQT + 32, r + 32);
+        tmem_ld_wait();
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t r[64];
-          tmem_ld32(trow + L::COL_DP + 64 * half, r);
-          tmem_ld32(trow + L::COL_DP + 64 * half + 32, r + 32);
-          tmem_ld_wait();
+        for (int c = 0; c < 64; ++c) reg_fence(r[c]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_SLOTFREE + s));
+        // The previous tile's bulk reduce must have read the staging tile before
+        // it is rewritten; that wait comes only now, after the TMEM slot was
+        // released, so the next S^T / dP^T never waits on the reduction.
+        if (leader && pending) {
+          bulk_wait_group_read0();
+          mbar_arrive(bar(L::B_DQSFREE));
+          pending = false;
+        }
+        // staging tile [query c][d]: a warp writes 32 consecutive floats per row
+        if (n > 0 && !ra_wait_warp(bar(L::B_DQSFREE), (n - 1) & 1, abort_flag)) break;
+        if (d < D) {   // at D = 64 the upper half of dQ^T is the zero padding
 #pragma unroll
-          for (int c = 0; c < 64; ++c) reg_fence(r[c]);
-          if (half == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(L::B_SLOTFREE));
-          }
-          if (d < D) {   // at D = 64 the upper half of dQ^T is the zero padding
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (64 * half + c < rows) red_add_f32(dst + (int64_t)(64 * half + c) * D, __uint_as_float(r[c]) * p.scale);
-          }
+          for (int c = 0; c < 64; ++c) st_shared_f32(dqs + c * (D * 4) + d * 4, __uint_as_float(r[c]) * p.scale);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_DQSFULL));
+        if (leader) {
+          if (!ra_wait(bar(L::B_DQSFULL), n & 1, abort_flag)) break;
+          // rows past S fall outside the tensor map and are not written
+          tma_reduce_add_3d(&tm_dq, dqs, 0, q * L::QT, bh);
+          bulk_commit_group();
+          pending = true;
         }
       }
     }
+    if (leader && pending) bulk_wait_group0();
   }
 
   // ------------------------------------------------------------ teardown

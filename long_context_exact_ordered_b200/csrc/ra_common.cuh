@@ -269,9 +269,9 @@ __device__ __forceinline__ int32_t step_iter_next_warp(StepKvIter& it, int4& km)
 // Backward direction of the same ring: a key/value tile of ring block src
 // meets the query blocks (src + order[t]) mod P at steps t = 0, 1, ...
 // (rank r holds block (r - order[t]) mod P at step t).  QIter walks the
-// 128-row query tiles a key tile [k_first, k_last] must visit in that order,
+// 64-row query tiles a key tile [k_first, k_last] must visit in that order,
 // skipping tiles hidden from it by causal masking or disjoint segments.
-constexpr int kQTileBwd = 128;
+constexpr int kQTileBwd = 64;
 
 struct QIter {
   int32_t src;        // ring block of the key tile

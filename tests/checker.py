@@ -20,6 +20,11 @@ Tolerances (stated once, used by every parity test):
   that bound exceeds 1e-2.  For those cases an element passes when its
   excess over half a bf16 ulp is within max(1e-2, that bound); the mean-abs
   bound stays 1e-3.  Every other case uses the plain bf16 rule.
+* the blockwise feed-forward network (no tolerance stated for it): its bf16
+  output y is O(1), so rounding it alone averages ~ulp/4 ~ 2e-3; its hidden
+  layer is rounded to bf16 between the two products.  Rule: excess over half
+  a bf16 ulp within max(1e-2, the hidden layer's rounding bound) per element,
+  and the mean of that excess <= 1e-3.
 """
 
 from __future__ import annotations
@@ -64,12 +69,17 @@ class Cmp:
                 f"max_excess={self.max_excess:.3e} mean_abs={self.mean_abs:.3e} n={self.n}")
 
 
-def compare(gpu, ref, kind="bf16", max_abs=None, mean_abs=None, rounding_bound=None) -> Cmp:
+def compare(gpu, ref, kind="bf16", max_abs=None, mean_abs=None, rounding_bound=None, mean_of="raw") -> Cmp:
     """Compare arrays; ``kind`` is "bf16" (half-ulp excess rule) or "f32".
 
     ``rounding_bound`` (bf16 only): an array like ``ref`` from
     ``operand_rounding_bound``; the allowed excess of each element is then
-    max(max_abs, rounding_bound) instead of max_abs."""
+    max(max_abs, rounding_bound) instead of max_abs.  ``mean_of`` (bf16
+    only): "raw" applies the mean-abs bound to the raw error (the attention
+    rule); "excess" applies it to the excess over half a bf16 ulp, for
+    outputs with no stated tolerance whose typical magnitude is O(1), where
+    the output rounding alone averages about ulp/4 (the feed-forward
+    network)."""
     g = np.asarray(gpu, dtype=np.float64)
     r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (g.shape, r.shape)
@@ -91,6 +101,9 @@ def compare(gpu, ref, kind="bf16", max_abs=None, mean_abs=None, rounding_bound=N
             rule = f"bf16(excess<=max({lim:g}, operand rounding bound), mean<={mlim:g})"
         over = excess - allowed
         mex = float(excess.max()) if n else 0.0
+        if mean_of == "excess":
+            mean = float(excess.mean()) if n else 0.0
+            rule = rule.replace("mean<=", "mean excess<=")
         ok = (float(over.max()) <= 0.0 if n else True) and mean <= mlim
     else:
         lim = F32_MAX_ABS if max_abs is None else max_abs

@@ -66,6 +66,13 @@ def test_compare_planted_errors():
     assert compare(plant(1, hu + 0.04), ref, "bf16", rounding_bound=bound).ok
     assert not compare(plant(1, hu + 0.06), ref, "bf16", rounding_bound=bound).ok
     assert not compare(plant(0, 0.04), ref, "bf16", rounding_bound=bound).ok
+    # the mean bound on the excess over half an ulp (feed-forward rule): O(1) values
+    # rounded to bf16 pass, an added bias of 2e-3 beyond half an ulp does not
+    big = np.linspace(1.0, 1.99, 1000)
+    rounded = torch.from_numpy(big).to(torch.bfloat16).double().numpy()
+    assert not compare(rounded, big, "bf16").ok                       # raw mean ~ ulp/4 > 1e-3
+    assert compare(rounded, big, "bf16", mean_of="excess").ok
+    assert not compare(big + bf16_half_ulp(big) + 2e-3, big, "bf16", mean_of="excess").ok
     # fp32 rule: raw max-abs
     assert compare(ref + 9e-6, ref, "f32").ok and not compare(plant(2, 1.1e-5), ref, "f32").ok
 
