@@ -24,10 +24,12 @@
 // query columns 0-31 and 32-63 of each tile: P^T, dS^T, then dK resp. dV in
 // the epilogue), warps 8-11 dQ readout (thread = head-dim lane d of dQ^T).
 // TMEM (512 columns): two 128-column slots, then dK [256,256+D), dV [256+D,256+2D).
-// Query tile n uses slot n % 2: S^T -> [0,64), dP^T -> [64,128); the softmax
-// group overwrites [0,32) with P^T and [32,64) with dS^T (bf16), and dQ^T(n)
-// lands in [64,128) once dP^T has been read.  A slot is reused two tiles
-// later, after the readout group has taken dQ^T out of it.
+// Query tile n uses slot n % 2: S^T -> [0,64), dP^T -> [64,128); softmax
+// group h overwrites its own S^T columns [32h, 32h+32) with P^T ([32h,
+// 32h+16)) and dS^T ([32h+16, 32h+32), bf16 pairs), so no group writes a
+// column the other still has to read, and dQ^T(n) lands in [64,128) once
+// dP^T has been read.  A slot is reused two tiles later, after the readout
+// group has taken dQ^T out of it.
 //
 // Overlap: with two slots the "head" products of tile n+1 (S^T, dP^T) are
 // computed while the softmax groups work on tile n; the issue order is given
@@ -88,7 +90,10 @@ struct BwdLayout {
   static constexpr int SMEM_ALLOC = BYTES + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t SLOT_COLS = 128;
-  static constexpr uint32_t SLOT_ST = 0, SLOT_DPT = 64, SLOT_PT = 0, SLOT_DST = 32, SLOT_DQT = 64;
+  // Softmax group h (query columns [32h, 32h+32)) writes its P^T into S^T
+  // columns [32h, 32h+16) and its dS^T into [32h+16, 32h+32): only columns of
+  // its own rows and queries that it has already read.
+  static constexpr uint32_t SLOT_ST = 0, SLOT_DPT = 64, SLOT_PT = 0, SLOT_DST = 16, SLOT_DQT = 64;
   static constexpr uint32_t COL_DK = 256, COL_DV = 256 + D;
   static constexpr int THREADS = 512;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
@@ -278,7 +283,8 @@ __global__ void __launch_bounds__(512, 1)
         const uint64_t b_desc = smem_desc_sw128(b_base, L::Q_CHUNK, 1024);
 #pragma unroll
         for (int kk = 0; kk < L::QT / 16; ++kk)
-          mma_ts_w(d_tmem, a_tmem + kk * 8, b_desc + kk * (2048 >> 4), IDESC_KV, (acc || kk > 0) ? 1u : 0u);
+          mma_ts_w(d_tmem, a_tmem + 32 * (kk / 2) + 8 * (kk % 2), b_desc + kk * (2048 >> 4), IDESC_KV,
+                   (acc || kk > 0) ? 1u : 0u);
       };
       auto issue_dq = [&](uint32_t d_tmem, uint32_t ds_base) {
         const uint64_t b_desc = smem_desc_sw128(ds_base, L::DS_BYTES, 1024);
@@ -437,8 +443,8 @@ __global__ void __launch_bounds__(512, 1)
           dd[c >> 1] = pack_bf16x2(ds0, ds1);
         }
         // P^T and dS^T (bf16, two per column) into this slot's first half.
-        tmem_st16(slot + L::SLOT_PT + c0 / 2, pp);
-        tmem_st16(slot + L::SLOT_DST + c0 / 2, dd);
+        tmem_st16(slot + L::SLOT_PT + c0, pp);
+        tmem_st16(slot + L::SLOT_DST + c0, dd);
         // dS^T into shared memory for dQ^T = K^T dS^T (MN-major, 128-byte swizzle):
         // key row `row` is one 128-byte line; 16-byte chunk c lands at c ^ (row % 8).
         const uint32_t line = sbase + L::OFF_DS + s * L::DS_BYTES + row * 128;

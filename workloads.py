@@ -18,6 +18,7 @@ causal128k     1   32  128  131072     8  512    1       bf16 N(0,1) (+dO)
 causal64k      1   32  128  65536      8  512    1       bf16 N(0,1) + dO, fwd+bwd
 causal1m       1   32  128  1048576    8  512    1       bf16 N(0,1)/sqrt(128)
 causal16k      1   32  128  16384      8  512    1       bf16 N(0,1) + dO (profiling)
+causal32k      1   32  128  32768      8  512    1       bf16 N(0,1) + dO (profiling)
 causal128k_c64 1  32  128  131072     8  512    64      bf16 N(0,1) + dO, block-causal
 causal128k_c512 1 32  128  131072     8  512    512     bf16 N(0,1) + dO, block-causal
 =============  ==  ==  ===  =========  =  =====  ======  ========================
@@ -75,6 +76,8 @@ WORKLOADS = {
                  description="million-token causal forward"),
         Workload("causal16k", 1, 32, 128, 16384, 8, 512, 1, backward=True, seed=1006,
                  description="profiling size: causal forward+backward, every input larger than L2"),
+        Workload("causal32k", 1, 32, 128, 32768, 8, 512, 1, backward=True, seed=1007,
+                 description="profiling size: causal forward+backward, second point of DRAM scaling"),
         Workload("causal128k_c64", 1, 32, 128, 131072, 8, 512, 64, backward=True, seed=1003,
                  description="block-causal (causal_block_size 64) forward+backward at 128K tokens"),
         Workload("causal128k_c512", 1, 32, 128, 131072, 8, 512, 512, backward=True, seed=1003,
