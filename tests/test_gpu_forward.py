@@ -85,11 +85,39 @@ def make_small(D, S, P, c, segments, bias, B, H, dtype="bf16", seed=11):
         b = torch.randn((B, S), generator=g)
         b[:, torch.randint(0, S, (S // 5,), generator=g)] = float("-inf")
         inp["bias"] = b.to(dev())
+    elif bias == "ramp":
+        # scores grow along the keys by ~9 (log2 units) per half tile: the
+        # softmax reference must move inside every key tile
+        inp["bias"] = (0.1 * torch.arange(S, dtype=torch.float32)).expand(B, S).contiguous().to(dev())
     return w, inp
 
 
 @pytest.mark.parametrize("case", SMALL, ids=lambda c: "D{}-S{}-P{}-c{}-{}-{}-B{}H{}".format(*c))
 def test_bf16_small_full_parity(case):
+    w, inp = make_small(*case)
+    o, lse = run(inp, w)
+    ro, rl = oracle_full(inp, w.causal_block_size)
+    res = compare(to64(o), ro, "bf16")
+    assert res.ok, str(res)
+    assert_lse(to64(lse), rl, LSE_BF16)
+    assert ra.device_status() == 0
+
+
+RAMP = [
+    # D,   S,    P, c,    segments, bias,   B, H
+    (64, 1024, 2, 1, None, "ramp", 1, 2),
+    (64, 1024, 2, None, None, "ramp", 1, 2),
+    (128, 1024, 2, 1, None, "ramp", 1, 2),
+    (64, 1024, 4, 1, "packed", "ramp", 1, 2),
+]
+
+
+@pytest.mark.parametrize("case", RAMP, ids=lambda c: "D{}-S{}-P{}-c{}-{}-{}-B{}H{}".format(*c))
+def test_reference_moves_inside_tiles(case):
+    """Scores that keep growing along the keys move the softmax's running
+    reference inside key tiles (the head-dim-64 kernel's recomputation of a
+    half tile after the reference moves, in either half, and the O rescale
+    that waits for the PV in flight)."""
     w, inp = make_small(*case)
     o, lse = run(inp, w)
     ro, rl = oracle_full(inp, w.causal_block_size)

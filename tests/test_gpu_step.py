@@ -40,6 +40,10 @@ def make(D, S, P, c, segments, bias, B, H, seed=51):
         b = torch.randn((B, S), generator=g)
         b[:, torch.randint(0, S, (S // 5,), generator=g)] = float("-inf")
         inp["bias"] = b.to(dev())
+    elif bias == "ramp":
+        # scores grow along the keys by ~9 (log2 units) per half tile: the
+        # softmax reference must move inside every key tile
+        inp["bias"] = (0.1 * torch.arange(S, dtype=torch.float32)).expand(B, S).contiguous().to(dev())
     return w, inp
 
 
@@ -86,6 +90,7 @@ CASES = [
     (128, 640, 5, 1, "packed", "neginf", 2, 2),   # segments and a bias with masked keys
     (64, 768, 2, None, None, "neginf", 1, 3),
     (128, 8192, 2, 1, "packed", None, 1, 2),      # 4096-token blocks: many tiles per step
+    (64, 1024, 4, 1, None, "ramp", 1, 2),         # the softmax reference moves inside key tiles
 ]
 
 
