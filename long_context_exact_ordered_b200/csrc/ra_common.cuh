@@ -72,6 +72,8 @@ struct KvIter {
   int32_t q_seg_min, q_seg_max;
   int32_t use_seg, use_bias;
   const int4* meta;   // this batch row's tile metadata, or null
+  uint32_t win;       // warp iterator: visible tiles of the window at win_base not yet returned
+  int32_t win_base;
 };
 
 RA_HD void kv_iter_init(KvIter& it, const RingDesc& rd, int64_t q_first, int64_t q_last, const int4* meta_b,
@@ -85,6 +87,8 @@ RA_HD void kv_iter_init(KvIter& it, const RingDesc& rd, int64_t q_first, int64_t
   it.meta = (use_seg || use_bias) ? meta_b : nullptr;
   it.use_seg = use_seg;
   it.use_bias = use_bias;
+  it.win = 0;
+  it.win_base = 0;
   it.q_seg_min = 0x7fffffff;
   it.q_seg_max = -0x7fffffff - 1;
   if (use_seg) {
@@ -131,24 +135,26 @@ RA_HD int32_t kv_iter_next(KvIter& it, const RingDesc& rd) {
 
 #ifdef __CUDACC__
 // kv_iter_next for a converged warp whose lanes all hold the same iterator:
-// the lanes test 32 candidate tiles at once, so a run of skipped tiles costs
-// one metadata round trip per 32 tiles instead of one per tile.  Returns the
-// same sequence as kv_iter_next.
+// the lanes test 32 candidate tiles at once and the warp keeps the ballot, so
+// both skipped and visible tiles cost one metadata round trip per 32 tiles
+// instead of one per tile.  Returns the same sequence as kv_iter_next.
 __device__ __forceinline__ int32_t kv_iter_next_warp(KvIter& it, const RingDesc& rd) {
   const int lane = threadIdx.x & 31;
   while (true) {
     if (!it.meta) {
       if (it.tile < it.tile_end) return it.tile++;
     } else {
-      while (it.tile < it.tile_end) {
-        const int32_t t = it.tile + lane;
-        const bool vis = t < it.tile_end && kv_tile_visible(it, load_meta(it.meta + t));
-        const unsigned hit = __ballot_sync(0xffffffffu, vis);
-        if (hit) {
-          const int32_t first = it.tile + __ffs(hit) - 1;
-          it.tile = first + 1;
+      while (true) {
+        if (it.win) {   // the window's visibility is known: no round trip
+          const int32_t first = it.win_base + __ffs(it.win) - 1;
+          it.win &= it.win - 1;
           return first;
         }
+        if (it.tile >= it.tile_end) break;
+        const int32_t t = it.tile + lane;
+        const bool vis = t < it.tile_end && kv_tile_visible(it, load_meta(it.meta + t));
+        it.win = __ballot_sync(0xffffffffu, vis);
+        it.win_base = it.tile;
         it.tile += 32;
       }
     }
@@ -282,6 +288,8 @@ struct QIter {
   int32_t k_seg_min, k_seg_max;
   int32_t use_seg;
   const int4* meta;   // 128-token tile metadata of this batch row, or null
+  uint32_t win;       // warp iterator: visible tiles of the window at win_base not yet returned
+  int32_t win_base;
 };
 
 RA_HD void q_iter_init(QIter& it, const RingDesc& rd, int64_t k_first, const int4* meta_b, bool use_seg) {
@@ -293,6 +301,8 @@ RA_HD void q_iter_init(QIter& it, const RingDesc& rd, int64_t k_first, const int
   it.q_min = (int32_t)(i_min / kQTileBwd);
   it.use_seg = use_seg;
   it.meta = use_seg ? meta_b : nullptr;
+  it.win = 0;
+  it.win_base = 0;
   it.k_seg_min = 0;
   it.k_seg_max = 0;
   if (use_seg) {
@@ -338,15 +348,17 @@ __device__ __forceinline__ int32_t q_iter_next_warp(QIter& it, const RingDesc& r
     if (!it.meta) {
       if (it.tile < it.tile_end) return it.tile++;
     } else {
-      while (it.tile < it.tile_end) {
-        const int32_t q = it.tile + lane;
-        const bool vis = q < it.tile_end && q_tile_visible(it, q);
-        const unsigned hit = __ballot_sync(0xffffffffu, vis);
-        if (hit) {
-          const int32_t first = it.tile + __ffs(hit) - 1;
-          it.tile = first + 1;
+      while (true) {
+        if (it.win) {
+          const int32_t first = it.win_base + __ffs(it.win) - 1;
+          it.win &= it.win - 1;
           return first;
         }
+        if (it.tile >= it.tile_end) break;
+        const int32_t q = it.tile + lane;
+        const bool vis = q < it.tile_end && q_tile_visible(it, q);
+        it.win = __ballot_sync(0xffffffffu, vis);
+        it.win_base = it.tile;
         it.tile += 32;
       }
     }
