@@ -403,7 +403,9 @@ __global__ void __launch_bounds__(512, 1)
           const int64_t cmax64 = S - (q0 + c0);                    // valid iff c < cmax
           const int cmax = row_valid ? (cmax64 > 32 ? 32 : (cmax64 < 0 ? 0 : (int)cmax64)) : 0;
           uint32_t vb = ~0u;
-          if (need_seg) {
+          if (need_seg && qm.x == qm.y) {
+            vb = my_seg == qm.x ? ~0u : 0u;   // every query of the tile is in segment qm.x
+          } else if (need_seg) {
             const int32_t* sp = p.seg + b * p.seg_sb;
             vb = 0;
 #pragma unroll

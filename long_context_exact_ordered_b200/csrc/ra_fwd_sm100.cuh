@@ -601,7 +601,11 @@ __global__ void __launch_bounds__(384, 1)
         const int64_t lim64 = jmax - k0;
         const int lim = lim64 < -1 ? -1 : (lim64 > 127 ? 127 : (int)lim64);
         uint32_t vb[4] = {~0u, ~0u, ~0u, ~0u};   // segment match bits, 32 keys per word
-        if (use_seg) {
+        if (use_seg && km.x == km.y) {
+          // every key of the tile is in segment km.x: the row sees all or none
+          const uint32_t all = my_seg == km.x ? ~0u : 0u;
+          vb[0] = vb[1] = vb[2] = vb[3] = all;
+        } else if (use_seg) {
           const int32_t* sp = segk + bk * segk_sb;
 #pragma unroll
           for (int w = 0; w < 4; ++w) {
