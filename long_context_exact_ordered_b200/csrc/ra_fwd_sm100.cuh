@@ -71,41 +71,16 @@ struct FwdLayout {
   static constexpr int B_KEMPTY = B_KFULL + KS;
   static constexpr int B_VFULL = B_KEMPTY + KS;
   static constexpr int B_VEMPTY = B_VFULL + VS;
-  // Head dim 64 leaves TMEM room for three S slots shared by the two query
-  // tiles in rotation (S_q(n) in slot (2n + q) mod 3), so each S is computed
-  // a tile ahead of the softmax that reads it; head dim 128 has one S slot
-  // per query tile.
-  static constexpr bool ROT = D == 64;
-  static constexpr int NSLOT = ROT ? 3 : 2;
-  static constexpr int B_SFULL = B_VEMPTY + VS;      // [NSLOT]
-  // Per query tile q: P of keys 0-63 / 64-127 written [q][half], PV(n)
-  // done [q], its first key half done [q].  With rotating slots a softmax
-  // warp can run one tile ahead of the issuer (never two), so each event
-  // then gets a barrier per key-tile parity, [..][n & 1], and the phase a
-  // wait names is never two phases away from the barrier's state.
-  static constexpr int B_PFULL = B_SFULL + NSLOT;    // [2][2][2]
-  static constexpr int B_PVDONE = B_PFULL + 8;       // [2][2]
-  static constexpr int B_PVH0 = B_PVDONE + 4;        // [2][2]
-  static constexpr int B_DRAIN = B_PVH0 + 4;         // issuer's final commit
+  static constexpr int B_SFULL = B_VEMPTY + VS;      // [2]
+  static constexpr int B_PFULL = B_SFULL + 2;        // [2][2]: P of keys 0-63 / 64-127 written, per query tile
+  static constexpr int B_PVDONE = B_PFULL + 4;       // [2]
+  static constexpr int B_DRAIN = B_PVDONE + 2;       // issuer's final commit
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;   // tmem slot, abort flag
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t COL_O0 = ROT ? 0 : 256, COL_O1 = COL_O0 + D;
-  static constexpr uint32_t COL_SLOT0 = ROT ? 128 : 0;   // slot s at COL_SLOT0 + 128 s
-  // S slot of query tile q at its n-th key tile, and the phase parity of that
-  // slot's barrier for this use.
-  __device__ static __forceinline__ int slot(int q, int n) { return ROT ? (2 * n + q) % 3 : q; }
-  __device__ static __forceinline__ int pfull(int q, int half, int n) {
-    return ROT ? B_PFULL + 4 * q + 2 * half + (n & 1) : B_PFULL + 2 * q + half;
-  }
-  __device__ static __forceinline__ int pvdone(int q, int n) { return ROT ? B_PVDONE + 2 * q + (n & 1) : B_PVDONE + q; }
-  __device__ static __forceinline__ int pvh0(int q, int n) { return ROT ? B_PVH0 + 2 * q + (n & 1) : B_PVH0 + q; }
-  __device__ static __forceinline__ uint32_t ev_parity(int n) { return (uint32_t)(ROT ? (n >> 1) & 1 : n & 1); }
-  __device__ static __forceinline__ uint32_t slot_parity(int q, int n) {
-    return ROT ? (uint32_t)(((2 * n + q) / 3) & 1) : (uint32_t)(n & 1);
-  }
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
   // Register split (setmaxnreg): warpgroup 0 (producer, MMA issuer) gives up
   // registers to the two softmax warpgroups.  The host checks
   // 128*REGS_LOW + 256*REGS_HIGH <= 384 * (registers per thread at launch)
@@ -180,70 +155,6 @@ struct FwdTiles<true> {
 };
 
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
-constexpr float kSumLimit = 256.0f;         // 2^kRescaleThreshold
-
-// Softmax helpers of the tensor-core forward (one thread = one query row).
-// They index the row's scores x[] with compile-time offsets only, so the
-// scores and the TMEM load destinations stay in registers.
-
-// max of x[C0 .. 127]
-template <int C0>
-__device__ __forceinline__ float fwd_row_max(const float* x) {
-  float mx0 = fmaxf(x[C0], x[C0 + 1]), mx1 = fmaxf(x[C0 + 2], x[C0 + 3]);
-#pragma unroll
-  for (int c = C0 + 4; c < 128; c += 4) {
-    mx0 = fmax3(mx0, x[c], x[c + 1]);
-    mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
-  }
-  return fmaxf(mx0, mx1);
-}
-
-// Moves the reference m_ref (log2 units) to mx when mx exceeds it by more
-// than kRescaleThreshold; returns the factor that earlier sums must take.
-__device__ __forceinline__ float fwd_move_ref(float& m_ref, float mx) {
-  if (!(mx > m_ref + kRescaleThreshold)) return 1.f;
-  const float alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
-  m_ref = mx;
-  return alpha;
-}
-
-// O row *= alpha in TMEM (warp-collective; no PV into it may be in flight).
-template <int D>
-__device__ __forceinline__ void fwd_rescale_o(uint32_t tO_row, float alpha) {
-#pragma unroll
-  for (int c = 0; c < D; c += 32) {
-    uint32_t orow[32];
-    tmem_ld32(tO_row + c, orow);
-    tmem_ld_wait();
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      reg_fence(orow[e]);
-      orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
-    }
-    tmem_st32(tO_row + c, orow);
-  }
-}
-
-// Exponentials 2^(x*sc - m_ref) of keys 64*HALF .. +63, packed as bf16
-// pairs into pk[32]; returns their fp32 sum.
-template <int HALF>
-__device__ __forceinline__ float fwd_exps_half(const float* x, float sc, float m_ref, uint32_t* pk) {
-  const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
-  float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-#pragma unroll
-  for (int c = 0; c < 64; c += 4) {
-    const int i = HALF * 64 + c;
-    float a0, a1, a2, a3;
-    ffma2(a0, a1, x[i], x[i + 1], sc, sc, nref, nref);
-    ffma2(a2, a3, x[i + 2], x[i + 3], sc, sc, nref, nref);
-    const float e0 = ex2_approx(a0), e1 = ex2_approx(a1), e2 = ex2_approx(a2), e3 = ex2_approx(a3);
-    fadd2(l0, l1, l0, l1, e0, e1);
-    fadd2(l2, l3, l2, l3, e2, e3);
-    pk[c >> 1] = pack_bf16x2(e0, e1);
-    pk[(c >> 1) + 1] = pack_bf16x2(e2, e3);
-  }
-  return (l0 + l1) + (l2 + l3);
-}
 
 template <int D, bool STEP>
 __global__ void __launch_bounds__(384, 1)
@@ -275,11 +186,11 @@ __global__ void __launch_bounds__(384, 1)
     mbar_init(bar(L::B_Q), 1);
     for (int i = 0; i < L::KS; ++i) { mbar_init(bar(L::B_KFULL + i), 1); mbar_init(bar(L::B_KEMPTY + i), 1); }
     for (int i = 0; i < L::VS; ++i) { mbar_init(bar(L::B_VFULL + i), 1); mbar_init(bar(L::B_VEMPTY + i), 1); }
-    for (int i = 0; i < L::NSLOT; ++i) mbar_init(bar(L::B_SFULL + i), 1);
-    for (int i = 0; i < 8; ++i) mbar_init(bar(L::B_PFULL + i), 4);   // one arrive per softmax warp
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(L::B_SFULL + i), 1);
+      mbar_init(bar(L::B_PFULL + 2 * i), 4);       // one arrive per softmax warp
+      mbar_init(bar(L::B_PFULL + 2 * i + 1), 4);
       mbar_init(bar(L::B_PVDONE + i), 1);
-      mbar_init(bar(L::B_PVH0 + i), 1);
     }
     mbar_init(bar(L::B_DRAIN), 1);
     *abort_flag = 0;
@@ -352,31 +263,24 @@ __global__ void __launch_bounds__(384, 1)
     {   // the whole warp runs the issuer; one elected lane issues (ptx.cuh)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+      const uint32_t tS[2] = {tmem + L::COL_S0, tmem + L::COL_S1};
       const uint32_t tO[2] = {tmem + L::COL_O0, tmem + L::COL_O1};
-      auto tS = [&](int sl) { return tmem + L::COL_SLOT0 + 128u * (uint32_t)sl; };
-      // Shared-memory descriptors are built once; each MMA adds a constant to
-      // the start-address field (address >> 4 in the low 14 bits; every
-      // address here stays below 2^18, so the add never carries out of it).
-      // The issuer shares its sub-partition with two softmax warps, so every
-      // instruction it saves shortens the softmax -> MMA -> softmax chain.
-      const uint64_t q_desc0 = smem_desc_sw128(sbase + L::OFF_Q, 16, 1024);
-      const uint64_t k_desc0 = smem_desc_sw128(sbase + L::OFF_K, 16, 1024);
-      const uint64_t v_desc0 = smem_desc_sw128(sbase + L::OFF_V, L::CHUNK_BYTES, 1024);
-      auto issue_s = [&](int qt, int ks, int sl) {
-        const uint64_t qd = q_desc0 + (uint32_t)(qt * (L::TILE_BYTES >> 4));
-        const uint64_t kd = k_desc0 + (uint32_t)(ks * (L::TILE_BYTES >> 4));
+      auto issue_s = [&](int qt, int ks) {
+        const uint32_t qa = sbase + L::OFF_Q + qt * L::TILE_BYTES;
+        const uint32_t ka = sbase + L::OFF_K + ks * L::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * L::CHUNK_BYTES + (kk % 4) * 32) >> 4;
-          mma_ss_w(tS(sl), qd + off, kd + off, IDESC_S, kk > 0);
+          const uint32_t off = (kk / 4) * L::CHUNK_BYTES + (kk % 4) * 32;
+          mma_ss_w(tS[qt], smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(ka + off, 16, 1024), IDESC_S,
+                 kk > 0);
         }
       };
-      auto issue_pv = [&](int qt, int vs, int key_half, bool acc, int sl) {   // keys 64*key_half .. +63
-        const uint64_t vd = v_desc0 + (uint32_t)(vs * (L::TILE_BYTES >> 4));
+      auto issue_pv = [&](int qt, int vs, int key_half, bool acc) {   // keys 64*key_half .. +63
+        const uint32_t va = sbase + L::OFF_V + vs * L::TILE_BYTES;
 #pragma unroll
         for (int k = 0; k < kTile / 32; ++k) {
           const int kk = key_half * (kTile / 32) + k;
-          mma_ts_w(tO[qt], tS(sl) + kk * 8, vd + (uint32_t)(kk * (2048 >> 4)), IDESC_PV,
+          mma_ts_w(tO[qt], tS[qt] + kk * 8, smem_desc_sw128(va + kk * 2048, L::CHUNK_BYTES, 1024), IDESC_PV,
                    (acc || k > 0) ? 1u : 0u);
         }
       };
@@ -384,78 +288,13 @@ __global__ void __launch_bounds__(384, 1)
       tiles.init(p, b, q0, meta_b, use_seg, use_bias);
       int32_t t = tiles.next(p);
       bool ok = ra_wait_warp(bar(L::B_Q), 0, abort_flag);
-      if constexpr (L::ROT) {
-        // Order: S0(n+1) is already issued when the loop reaches n; PV0(n),
-        // S1(n+1) into the slot PV0(n) frees, PV1(n), S0(n+2) into the slot
-        // PV1(n) frees.  The tensor pipe executes this thread's MMAs in
-        // issue order, so an S is issued right behind the PV that reads the
-        // P it overwrites.
-        bool has1 = false, has2 = false;   // key tiles n+1, n+2 exist
-        if (ok && t >= 0) {
-          ok = ra_wait_warp(bar(L::B_KFULL + 0), 0, abort_flag);
-          if (ok) {
-            tc_fence_after();
-            issue_s(0, 0, L::slot(0, 0));
-            mma_commit_w(bar(L::B_SFULL + L::slot(0, 0)));
-            issue_s(1, 0, L::slot(1, 0));
-            mma_commit_w(bar(L::B_SFULL + L::slot(1, 0)));
-            mma_commit_w(bar(L::B_KEMPTY + 0));
-            has1 = tiles.next(p) >= 0;
-            if (has1) {
-              ok = ra_wait_warp(bar(L::B_KFULL + 1 % L::KS), (1 / L::KS) & 1, abort_flag);
-              if (ok) {
-                issue_s(0, 1 % L::KS, L::slot(0, 1));
-                mma_commit_w(bar(L::B_SFULL + L::slot(0, 1)));
-              }
-              has2 = tiles.next(p) >= 0;
-            }
-          }
-          for (int n = 0; ok; ++n) {
-            const int vs = n % L::VS, ks1 = (n + 1) % L::KS, ks2 = (n + 2) % L::KS;
-            const uint32_t ph = L::ev_parity(n);
-            if (!(ok = ra_wait_warp(bar(L::B_VFULL + vs), (n / L::VS) & 1, abort_flag))) break;
-            // query tile 0; PV in two halves of the keys: the first runs while
-            // the softmax still computes P for the second
-            if (!(ok = ra_wait_warp(bar(L::pfull(0, 0, n)), ph, abort_flag))) break;
-            tc_fence_after();
-            issue_pv(0, vs, 0, n > 0, L::slot(0, n));
-            mma_commit_w(bar(L::pvh0(0, n)));
-            if (!(ok = ra_wait_warp(bar(L::pfull(0, 1, n)), ph, abort_flag))) break;
-            tc_fence_after();
-            issue_pv(0, vs, 1, true, L::slot(0, n));
-            mma_commit_w(bar(L::pvdone(0, n)));
-            if (has1) {   // K(n+1) landed before S0(n+1) was issued
-              issue_s(1, ks1, L::slot(1, n + 1));
-              mma_commit_w(bar(L::B_SFULL + L::slot(1, n + 1)));
-              mma_commit_w(bar(L::B_KEMPTY + ks1));
-            }
-            // query tile 1
-            if (!(ok = ra_wait_warp(bar(L::pfull(1, 0, n)), ph, abort_flag))) break;
-            tc_fence_after();
-            issue_pv(1, vs, 0, n > 0, L::slot(1, n));
-            mma_commit_w(bar(L::pvh0(1, n)));
-            if (!(ok = ra_wait_warp(bar(L::pfull(1, 1, n)), ph, abort_flag))) break;
-            tc_fence_after();
-            issue_pv(1, vs, 1, true, L::slot(1, n));
-            mma_commit_w(bar(L::pvdone(1, n)));
-            mma_commit_w(bar(L::B_VEMPTY + vs));
-            if (has2) {
-              if (!(ok = ra_wait_warp(bar(L::B_KFULL + ks2), ((n + 2) / L::KS) & 1, abort_flag))) break;
-              issue_s(0, ks2, L::slot(0, n + 2));
-              mma_commit_w(bar(L::B_SFULL + L::slot(0, n + 2)));
-            }
-            if (!has1) break;
-            has1 = has2;
-            has2 = has2 && tiles.next(p) >= 0;
-          }
-        }
-      } else if (ok && t >= 0) {
+      if (ok && t >= 0) {
         ok = ra_wait_warp(bar(L::B_KFULL + 0), 0, abort_flag);
         if (ok) {
           tc_fence_after();
-          issue_s(0, 0, 0);
+          issue_s(0, 0);
           mma_commit_w(bar(L::B_SFULL + 0));
-          issue_s(1, 0, 1);
+          issue_s(1, 0);
           mma_commit_w(bar(L::B_SFULL + 1));
           mma_commit_w(bar(L::B_KEMPTY + 0));
         }
@@ -463,37 +302,37 @@ __global__ void __launch_bounds__(384, 1)
           const int32_t tn = tiles.next(p);
           const bool last = tn < 0;
           const int vs = n % L::VS, ks1 = (n + 1) % L::KS;
-          const uint32_t ph = L::ev_parity(n);
+          const uint32_t ph = n & 1;
           if (!(ok = ra_wait_warp(bar(L::B_VFULL + vs), (n / L::VS) & 1, abort_flag))) break;
           // query tile 0
           // PV in two halves of the keys: the first runs while the softmax
           // still computes P for the second
-          if (!(ok = ra_wait_warp(bar(L::pfull(0, 0, n)), ph, abort_flag))) break;
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 0), ph, abort_flag))) break;
           tc_fence_after();
-          issue_pv(0, vs, 0, n > 0, 0);
-          if (!(ok = ra_wait_warp(bar(L::pfull(0, 1, n)), ph, abort_flag))) break;
+          issue_pv(0, vs, 0, n > 0);
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 1), ph, abort_flag))) break;
           tc_fence_after();
-          issue_pv(0, vs, 1, true, 0);
-          mma_commit_w(bar(L::pvdone(0, n)));
+          issue_pv(0, vs, 1, true);
+          mma_commit_w(bar(L::B_PVDONE + 0));
           if (!last) {
             // S0(n+1) overwrites the TMEM columns PV0(n) reads P0 from; the
             // tensor pipe executes this thread's MMAs in issue order, so it is
             // issued right behind PV0(n) without waiting for its completion.
             if (!(ok = ra_wait_warp(bar(L::B_KFULL + ks1), ((n + 1) / L::KS) & 1, abort_flag))) break;
-            issue_s(0, ks1, 0);
+            issue_s(0, ks1);
             mma_commit_w(bar(L::B_SFULL + 0));
           }
           // query tile 1
-          if (!(ok = ra_wait_warp(bar(L::pfull(1, 0, n)), ph, abort_flag))) break;
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 2), ph, abort_flag))) break;
           tc_fence_after();
-          issue_pv(1, vs, 0, n > 0, 1);
-          if (!(ok = ra_wait_warp(bar(L::pfull(1, 1, n)), ph, abort_flag))) break;
+          issue_pv(1, vs, 0, n > 0);
+          if (!(ok = ra_wait_warp(bar(L::B_PFULL + 3), ph, abort_flag))) break;
           tc_fence_after();
-          issue_pv(1, vs, 1, true, 1);
-          mma_commit_w(bar(L::pvdone(1, n)));
+          issue_pv(1, vs, 1, true);
+          mma_commit_w(bar(L::B_PVDONE + 1));
           mma_commit_w(bar(L::B_VEMPTY + vs));
           if (!last) {
-            issue_s(1, ks1, 1);
+            issue_s(1, ks1);
             mma_commit_w(bar(L::B_SFULL + 1));
             mma_commit_w(bar(L::B_KEMPTY + ks1));
           }
@@ -516,7 +355,7 @@ __global__ void __launch_bounds__(384, 1)
     const int64_t q_first = q0 + qt * kTile;
     const int64_t qrow = q_first + row;
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
-    const uint32_t tS_base = tmem + lane_off + L::COL_SLOT0;   // + 128 * slot
+    const uint32_t tS_row = tmem + lane_off + (qt ? L::COL_S1 : L::COL_S0);
     const uint32_t tO_row = tmem + lane_off + (qt ? L::COL_O1 : L::COL_O0);
     const int64_t qrow_c = qrow < S ? qrow : S - 1;
     const int my_seg = use_seg ? p.seg[b * p.seg_sb + qrow_c * p.seg_ss] : 0;
@@ -552,18 +391,10 @@ __global__ void __launch_bounds__(384, 1)
 #endif
     int n = 0;
     bool ok = true;
-    int32_t t = tiles.next(p);
-    while (t >= 0) {
+    for (int32_t t = tiles.next(p); t >= 0; t = tiles.next(p), ++n) {
       // the tile's metadata load is issued before the wait, so it lands while S is computed
       const int4 km = tiles.meta(t);
-      // With rotating S slots the softmax rarely waits for S, so the next
-      // tile's index (a warp-cooperative scan) is found while this tile is
-      // processed rather than after it.
-      int32_t t_next = -1;
-      if constexpr (L::ROT) t_next = tiles.next(p);
-      const int sl = L::slot(qt, n);
-      const uint32_t tS_row = tS_base + 128u * (uint32_t)sl;
-      if (!(ok = ra_wait_warp(bar(L::B_SFULL + sl), L::slot_parity(qt, n), abort_flag))) break;
+      if (!(ok = ra_wait_warp(bar(L::B_SFULL + qt), n & 1, abort_flag))) break;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld32(tS_row + 0, sr);
@@ -631,142 +462,66 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < 128; ++c) dbg_vis += x[c] != -INFINITY;
 #endif
-      const float sc = has_bias ? 1.f : p.scale_log2;   // x * sc is the score in log2 units
-      if constexpr (!L::ROT) {
-        // Head dim 128: the tile max first, then the exponentials.
-        // tile max (three-input max, two independent chains)
-        float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
+      // tile max (three-input max, two independent chains)
+      float mx0 = fmaxf(x[0], x[1]), mx1 = fmaxf(x[2], x[3]);
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmax3(mx0, x[c], x[c + 1]);
-          mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
-        }
-        const float mx = fmaxf(mx0, mx1) * sc;
-        const bool need = mx > m_ref + kRescaleThreshold;
-        float alpha = 1.f;
-        if (need) {
-          alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
-          m_ref = mx;
-          l *= alpha;
-        }
-        if (n > 0 && __any_sync(0xffffffffu, need)) {
-          // rescale this warp's O rows in TMEM (PV of the previous tile has completed:
-          // the commit that released S_q(n) covers it)
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t orow[32];
-            tmem_ld32(tO_row + c, orow);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              reg_fence(orow[e]);
-              orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
-            }
-            tmem_st32(tO_row + c, orow);
-          }
-        }
-        const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) {
-            const int i = half * 64 + c;
-            float a0, a1, a2, a3;
-            ffma2(a0, a1, x[i], x[i + 1], sc, sc, nref, nref);
-            ffma2(a2, a3, x[i + 2], x[i + 3], sc, sc, nref, nref);
-            const float e0 = ex2_approx(a0), e1 = ex2_approx(a1), e2 = ex2_approx(a2), e3 = ex2_approx(a3);
-            fadd2(l0, l1, l0, l1, e0, e1);
-            fadd2(l2, l3, l2, l3, e2, e3);
-            pk[c >> 1] = pack_bf16x2(e0, e1);
-            pk[(c >> 1) + 1] = pack_bf16x2(e2, e3);
-          }
-          tmem_st32(tS_row + half * 32, pk);
-          // P of this half of the keys is in TMEM: the MMA warp may start its half of PV
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(L::pfull(qt, half, n)));
-        }
-        l += (l0 + l1) + (l2 + l3);
-      } else {
-        // Exponentials are taken against the running reference m_ref without a
-        // tile max: a half tile whose sum of exponentials stays within
-        // 2^kRescaleThreshold has every term within it, which is all the
-        // reference must guarantee.  The tile max is computed only while a row
-        // has no finite score yet, or when a half's sum exceeds the limit (a
-        // larger score, or an overflow to inf): then the reference moves to
-        // the max, O and l are rescaled, and the half is recomputed.  Every
-        // branch below is warp-uniform (the O rescale is a warp-wide TMEM
-        // access).
-        // With rotating S slots, S_q(n) is issued before PV_q(n-1): a rescale
-        // of O waits for PV_q(n-1) explicitly.  With one slot per query tile
-        // the commit that released S_q(n) covers PV_q(n-1).
-        auto o_quiet = [&]() -> bool {
-          if (!L::ROT || n == 0) return true;
-          if (!ra_wait_warp(bar(L::pvdone(qt, n - 1)), L::ev_parity(n - 1), abort_flag)) return false;
-          tc_fence_after();
-          return true;
-        };
-        const bool exact_max = __any_sync(0xffffffffu, m_ref == -INFINITY);
-        if (exact_max) {
-          const float alpha = fwd_move_ref(m_ref, fwd_row_max<0>(x) * sc);
-          l *= alpha;
-          if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-            ok = o_quiet();
-            if (!ok) break;
-            fwd_rescale_o<D>(tO_row, alpha);
-          }
-        }
-        float lh0, lh1;
-        {
-          uint32_t pk[32];
-          lh0 = fwd_exps_half<0>(x, sc, m_ref, pk);
-          if (!exact_max && __any_sync(0xffffffffu, !(lh0 <= kSumLimit))) {
-            const float alpha = fwd_move_ref(m_ref, fwd_row_max<0>(x) * sc);
-            l *= alpha;
-            if (n > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-              ok = o_quiet();
-              if (!ok) break;
-              fwd_rescale_o<D>(tO_row, alpha);
-            }
-            lh0 = fwd_exps_half<0>(x, sc, m_ref, pk);
-          }
-          tmem_st32(tS_row, pk);
-          // P of this half of the keys is in TMEM: the MMA warp may start its half of PV
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(L::pfull(qt, 0, n)));
-        }
-        {
-          uint32_t pk[32];
-          lh1 = fwd_exps_half<1>(x, sc, m_ref, pk);
-          if (!exact_max && __any_sync(0xffffffffu, !(lh1 <= kSumLimit))) {
-            // PV(n) of the first key half may still be adding into O
-            if (!(ok = ra_wait_warp(bar(L::pvh0(qt, n)), L::ev_parity(n), abort_flag))) break;
-            tc_fence_after();
-            const float alpha = fwd_move_ref(m_ref, fwd_row_max<64>(x) * sc);
-            l *= alpha;
-            lh0 *= alpha;
-            if (__any_sync(0xffffffffu, alpha != 1.f)) fwd_rescale_o<D>(tO_row, alpha);
-            lh1 = fwd_exps_half<1>(x, sc, m_ref, pk);
-          }
-          tmem_st32(tS_row + 32, pk);
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(L::pfull(qt, 1, n)));
-        }
-        l += lh0 + lh1;
+      for (int c = 4; c < 128; c += 4) {
+        mx0 = fmax3(mx0, x[c], x[c + 1]);
+        mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
       }
-      if constexpr (!L::ROT) t_next = tiles.next(p);
-      t = t_next;
-      ++n;
+      const float sc = has_bias ? 1.f : p.scale_log2;   // x * sc is the score in log2 units
+      const float mx = fmaxf(mx0, mx1) * sc;
+      const bool need = mx > m_ref + kRescaleThreshold;
+      float alpha = 1.f;
+      if (need) {
+        alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx(m_ref - mx);
+        m_ref = mx;
+        l *= alpha;
+      }
+      if (n > 0 && __any_sync(0xffffffffu, need)) {
+        // rescale this warp's O rows in TMEM (PV of the previous tile has completed:
+        // the commit that released S_q(n) covers it)
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t orow[32];
+          tmem_ld32(tO_row + c, orow);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            reg_fence(orow[e]);
+            orow[e] = __float_as_uint(__uint_as_float(orow[e]) * alpha);
+          }
+          tmem_st32(tO_row + c, orow);
+        }
+      }
+      const float nref = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 64; c += 4) {
+          const int i = half * 64 + c;
+          float a0, a1, a2, a3;
+          ffma2(a0, a1, x[i], x[i + 1], sc, sc, nref, nref);
+          ffma2(a2, a3, x[i + 2], x[i + 3], sc, sc, nref, nref);
+          const float e0 = ex2_approx(a0), e1 = ex2_approx(a1), e2 = ex2_approx(a2), e3 = ex2_approx(a3);
+          fadd2(l0, l1, l0, l1, e0, e1);
+          fadd2(l2, l3, l2, l3, e2, e3);
+          pk[c >> 1] = pack_bf16x2(e0, e1);
+          pk[(c >> 1) + 1] = pack_bf16x2(e2, e3);
+        }
+        tmem_st32(tS_row + half * 32, pk);
+        // P of this half of the keys is in TMEM: the MMA warp may start its half of PV
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(L::B_PFULL + 2 * qt + half));
+      }
+      l += (l0 + l1) + (l2 + l3);
     }
     // ---------------------------------------------------------- epilogue
-    if (ok && n > 0) ok = ra_wait_warp(bar(L::pvdone(qt, n - 1)), L::ev_parity(n - 1), abort_flag);
+    if (ok && n > 0) ok = ra_wait_warp(bar(L::B_PVDONE + qt), (n - 1) & 1, abort_flag);
     n = __shfl_sync(0xffffffffu, n, 0);   // warp-uniform (lanes agree unless a wait gave up)
     tc_fence_after();
     if constexpr (STEP) {

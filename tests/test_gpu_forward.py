@@ -114,10 +114,9 @@ RAMP = [
 
 @pytest.mark.parametrize("case", RAMP, ids=lambda c: "D{}-S{}-P{}-c{}-{}-{}-B{}H{}".format(*c))
 def test_reference_moves_inside_tiles(case):
-    """Scores that keep growing along the keys move the softmax's running
-    reference inside key tiles (the head-dim-64 kernel's recomputation of a
-    half tile after the reference moves, in either half, and the O rescale
-    that waits for the PV in flight)."""
+    """Scores that keep growing along the keys (a bias ramp of ~9 log2 units
+    per half tile) move the softmax's running reference at every key tile,
+    so every tile takes the rescale of O and of the running sum."""
     w, inp = make_small(*case)
     o, lse = run(inp, w)
     ro, rl = oracle_full(inp, w.causal_block_size)

@@ -90,7 +90,7 @@ CASES = [
     (128, 640, 5, 1, "packed", "neginf", 2, 2),   # segments and a bias with masked keys
     (64, 768, 2, None, None, "neginf", 1, 3),
     (128, 8192, 2, 1, "packed", None, 1, 2),      # 4096-token blocks: many tiles per step
-    (64, 1024, 4, 1, None, "ramp", 1, 2),         # the softmax reference moves inside key tiles
+    (64, 1024, 4, 1, None, "ramp", 1, 2),         # the softmax reference moves at every key tile
 ]
 
 
