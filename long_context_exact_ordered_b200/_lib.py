@@ -118,6 +118,8 @@ def load_count() -> ctypes.CDLL:
         lib.ra_debug_ex2_rate.restype = ctypes.c_int
         lib.ra_debug_ex2_rate.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
                                           ctypes.c_void_p]
+        lib.ra_debug_bounds.restype = ctypes.c_int
+        lib.ra_debug_bounds.argtypes = [ctypes.POINTER(ctypes.c_uint64)]
         _count_lib = lib
     return _count_lib
 

@@ -1167,6 +1167,16 @@ int ra_debug_ex2_rate(int32_t iters, int32_t blocks, long long* cycles, float* s
   return cudaGetLastError() == cudaSuccess ? RA_OK : RA_ERR_CUDA;
 }
 
+int ra_debug_bounds(uint64_t* first_hit) {
+  if (!first_hit) return RA_ERR_NULL;
+  unsigned long long v = 0;
+  RA_TRY(cuda_fail(cudaMemcpyFromSymbol(&v, ra::g_ra_bounds_hit, sizeof(v)), "cudaMemcpyFromSymbol (index-check word)"));
+  const unsigned long long zero = 0;
+  RA_TRY(cuda_fail(cudaMemcpyToSymbol(ra::g_ra_bounds_hit, &zero, sizeof(zero)), "cudaMemcpyToSymbol (index-check word)"));
+  *first_hit = v;
+  return RA_OK;
+}
+
 int ra_debug_set_counts(int32_t* fwd_row_counts, int32_t* bwd_col_counts) {
   g_dbg_fwd_rows = fwd_row_counts;
   g_dbg_bwd_cols = bwd_col_counts;

@@ -172,6 +172,7 @@ __global__ void __launch_bounds__(512, 1)
   const int b = bh / p.H, h = bh % p.H;
   const int64_t k0 = (int64_t)kt * kTile;
   const int64_t S = p.rd.S;
+  if (!(RA_IN_RANGE(b, p.B, kSiteBwdUnit) && RA_IN_RANGE(h, p.H, kSiteBwdUnit))) return;   // debug build only
 
   auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::OFF_MISC);
@@ -248,8 +249,12 @@ __global__ void __launch_bounds__(512, 1)
               tma_load_4d(sbase + L::OFF_DO + st * L::Q_BYTES + c * L::Q_CHUNK, &tm_do, bar(L::B_QF + st), c * 64,
                           h, q0, b);
             }
-            bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES, lse_row + q0, L::QT * 4, bar(L::B_QF + st));
-            bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES + L::QT * 4, dl_row + q0, L::QT * 4, bar(L::B_QF + st));
+            // (an out-of-range row in the debug build skips the copies; the
+            // stage then never completes and its consumers' bounded waits give up)
+            if (RA_IN_RANGE(q0 + L::QT - 1, p.s_pad, kSiteBwdLseDelta)) {
+              bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES, lse_row + q0, L::QT * 4, bar(L::B_QF + st));
+              bulk_load(sbase + L::OFF_LD + st * L::LD_BYTES + L::QT * 4, dl_row + q0, L::QT * 4, bar(L::B_QF + st));
+            }
           }
           __syncwarp();
         }
@@ -352,9 +357,10 @@ __global__ void __launch_bounds__(512, 1)
     const int64_t jc = row_valid ? j : S - 1;
     const uint32_t lane_off = (uint32_t)(sub * 32) << 16;
     const uint32_t trow = tmem + lane_off;
-    const int my_seg = use_seg ? p.seg[b * p.seg_sb + jc * p.seg_ss] : 0;
+    const bool key_in = RA_IN_RANGE(jc, S, kSiteBwdKeyRow);
+    const int my_seg = use_seg && key_in ? p.seg[b * p.seg_sb + jc * p.seg_ss] : 0;
     float brow = 0.f;                                // bias of this key, log2 units
-    if (use_bias) brow = p.bias[b * p.bias_sb + jc * p.bias_ss] * kLog2e;
+    if (use_bias && key_in) brow = p.bias[b * p.bias_sb + jc * p.bias_ss] * kLog2e;
     const int32_t cbs = p.rd.cbs;
     const int64_t i_first = cbs > 0 ? (j / cbs) * (int64_t)cbs : 0;   // first query that can see key j
     // A query tile starting at q0 needs the causal mask iff q0 is before the
@@ -374,7 +380,8 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t slot = trow + s * L::SLOT_COLS;
         const int64_t q0 = (int64_t)q * L::QT;
         // the query tile's metadata load is issued before the waits, so it lands meanwhile
-        const int4 qm = meta_b ? load_meta(meta_b + q0 / kTile) : make_int4(0, 0, 3, 0);
+        const int4 qm = meta_b && RA_IN_RANGE(q0 / kTile, p.rd.ntiles, kSiteBwdQueryMeta) ? load_meta(meta_b + q0 / kTile)
+                                                                                      : make_int4(0, 0, 3, 0);
         if (!(ok = ra_wait_warp(bar(L::B_QF + st), (n / L::NS) & 1, abort_flag))) break;
         if (!(ok = ra_wait_warp(bar(L::B_SFULL + s), (n >> 1) & 1, abort_flag))) break;
         tc_fence_after();
@@ -411,7 +418,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               const int64_t i = q0 + c0 + c < S ? q0 + c0 + c : S - 1;
-              vb |= (uint32_t)(__ldg(sp + i * p.seg_ss) == my_seg) << c;
+              vb |= (uint32_t)(RA_IN_RANGE(i, S, kSiteBwdQuerySeg) && __ldg(sp + i * p.seg_ss) == my_seg) << c;
             }
           }
 #pragma unroll
@@ -453,7 +460,9 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int chunk = half * 4 + c;
-          st_shared_v4(line + ((chunk ^ (row & 7)) << 4), dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+          const uint32_t off = (uint32_t)row * 128 + ((chunk ^ (row & 7)) << 4);   // within this slot's dS^T buffer
+          if (RA_IN_RANGE(off + 15, L::DS_BYTES, kSiteBwdDsSmem))
+            st_shared_v4(line - (uint32_t)row * 128 + off, dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
         }
         fence_proxy_async_smem();
         tmem_st_wait();
@@ -494,7 +503,7 @@ __global__ void __launch_bounds__(512, 1)
           if (have) reg_fence(r[e]);
           else r[e] = 0u;
         }
-        if (row_valid && (have || n == 0)) {
+        if (row_valid && (have || n == 0) && key_in) {
           if (p.grad_bf16) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + off + c);
 #pragma unroll
@@ -553,7 +562,9 @@ __global__ void __launch_bounds__(512, 1)
         if (n > 0 && !ra_wait_warp(bar(L::B_DQSFREE), (n - 1) & 1, abort_flag)) break;
         if (d < D) {   // at D = 64 the upper half of dQ^T is the zero padding
 #pragma unroll
-          for (int c = 0; c < 64; ++c) st_shared_f32(dqs + c * (D * 4) + d * 4, __uint_as_float(r[c]) * p.scale);
+          for (int c = 0; c < 64; ++c)
+            if (RA_IN_RANGE(c * (D * 4) + d * 4 + 3, L::DQS_BYTES, kSiteBwdDqStaging))
+              st_shared_f32(dqs + c * (D * 4) + d * 4, __uint_as_float(r[c]) * p.scale);
         }
         fence_proxy_async_smem();
         __syncwarp();

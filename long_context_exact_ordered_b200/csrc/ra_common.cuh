@@ -46,6 +46,52 @@ enum : int32_t { kMetaAnyFinite = 1, kMetaAllZero = 2 };
 
 RA_HD int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Index checks of the debug build (-DRA_DEBUG_COUNT, libringattn_count.so).
+// Before each global or shared-memory access whose address a kernel computes
+// from indices (TMA copies excepted: the tensor maps bound those), the debug
+// build tests every index against its extent.  An index out of range skips the
+// access and records the first such event device-wide in g_ra_bounds_hit:
+// the site id (RaSite) in bits 48-63 and the index's low 48 bits below;
+// ra_debug_bounds() reads and clears it.  In the release build the test is
+// the constant true, and the indices are not even evaluated.
+enum RaSite : int {
+  kSiteFwdTileMeta = 1,   // forward: key-tile metadata (tile < ntiles)
+  kSiteFwdUnit,           // forward: batch row / head of the CTA's unit (b < B, h < H)
+  kSiteFwdQuerySeg,       // forward: query row's segment id (row < S)
+  kSiteFwdKeyBias,        // forward: key bias (key < Sk)
+  kSiteFwdKeySeg,         // forward: key segment id (key < Sk)
+  kSiteFwdStepState,      // ring step: running m, l and accumulator row (row < Sq)
+  kSiteFwdOut,            // forward: O row, LSE and visible-count stores (row < S)
+  kSiteBwdUnit,           // backward: batch row / head / key tile of the CTA (b < B, h < H)
+  kSiteBwdKeyRow,         // backward: key row's segment id, bias, dK / dV row (key < S)
+  kSiteBwdQueryMeta,      // backward: query tile's metadata (tile < ntiles)
+  kSiteBwdQuerySeg,       // backward: query segment ids (query < S)
+  kSiteBwdDsSmem,         // backward: dS^T shared-memory stores (byte offset < buffer)
+  kSiteBwdDqStaging,      // backward: dQ staging stores (byte offset < buffer)
+  kSiteBwdLseDelta,       // backward: LSE / Delta rows of a query tile (row + 64 <= padded rows)
+  kSiteIterMeta,          // tile iterators: key- and query-tile metadata (tile < ntiles)
+  kSiteStepKeys,          // ring-step iterator: visiting keys' segment ids / bias (key < Sk)
+  kSiteStepQueries,       // ring-step iterator: query segment ids (row < Sq)
+  kSiteTileMeta,          // tile metadata kernel: key reads and metadata write
+  kSiteBwdPre,            // backward preprocess: O, dO, LSE reads, Delta / LSE2 / dQ-accumulator writes
+  kSiteDqConvert,         // dQ conversion: accumulator read, dQ write
+  kSiteFinalize,          // finalize and LSE merge rows (row < B*S*H)
+  kSiteFfnOut,            // feed-forward GEMMs: output tile rows and columns
+};
+#if defined(RA_DEBUG_COUNT) && defined(__CUDACC__)
+__device__ unsigned long long g_ra_bounds_hit;
+#endif
+#if defined(RA_DEBUG_COUNT) && defined(__CUDA_ARCH__)
+__device__ __forceinline__ bool ra_in_range(long long i, long long n, int site) {
+  if (i >= 0 && i < n) return true;
+  atomicCAS(&g_ra_bounds_hit, 0ull, ((unsigned long long)site << 48) | ((unsigned long long)i & 0xFFFFFFFFFFFFull));
+  return false;
+}
+#define RA_IN_RANGE(i, n, site) ::ra::ra_in_range((long long)(i), (long long)(n), (site))
+#else
+#define RA_IN_RANGE(i, n, site) true
+#endif
+
 #if defined(__CUDA_ARCH__)
 RA_HD int4 load_meta(const int4* p) { return __ldg(p); }
 #else
@@ -93,6 +139,7 @@ RA_HD void kv_iter_init(KvIter& it, const RingDesc& rd, int64_t q_first, int64_t
   it.q_seg_max = -0x7fffffff - 1;
   if (use_seg) {
     for (int64_t qt = q_first / kTile; qt <= q_last / kTile; ++qt) {
+      if (!RA_IN_RANGE(qt, rd.ntiles, kSiteIterMeta)) break;
       int4 m = load_meta(meta_b + qt);
       it.q_seg_min = m.x < it.q_seg_min ? m.x : it.q_seg_min;
       it.q_seg_max = m.y > it.q_seg_max ? m.y : it.q_seg_max;
@@ -152,7 +199,8 @@ __device__ __forceinline__ int32_t kv_iter_next_warp(KvIter& it, const RingDesc&
         }
         if (it.tile >= it.tile_end) break;
         const int32_t t = it.tile + lane;
-        const bool vis = t < it.tile_end && kv_tile_visible(it, load_meta(it.meta + t));
+        const bool vis = t < it.tile_end && RA_IN_RANGE(t, rd.ntiles, kSiteIterMeta) &&
+                         kv_tile_visible(it, load_meta(it.meta + t));
         it.win = __ballot_sync(0xffffffffu, vis);
         it.win_base = it.tile;
         it.tile += 32;
@@ -191,7 +239,7 @@ __device__ __forceinline__ int4 step_tile_meta_warp(const StepKvIter& it, int32_
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int64_t j = (int64_t)t * kTile + lane * 4 + i;
-    if (j < it.Sk) {
+    if (j < it.Sk && RA_IN_RANGE(j, it.Sk, kSiteStepKeys)) {
       const int s = it.seg_k ? __ldg(it.seg_k + j * it.segk_ss) : 0;
       smin = s < smin ? s : smin;
       smax = s > smax ? s : smax;
@@ -218,6 +266,7 @@ __device__ __forceinline__ int2 step_q_seg_range_warp(const int32_t* seg_q, int6
   int smin = 0x7fffffff, smax = -0x7fffffff - 1;
   if (q_last > Sq - 1) q_last = Sq - 1;
   for (int64_t i = q_first + lane; i <= q_last; i += 32) {
+    if (!RA_IN_RANGE(i, Sq, kSiteStepQueries)) break;
     const int s = __ldg(seg_q + i * segq_ss);
     smin = s < smin ? s : smin;
     smax = s > smax ? s : smax;
@@ -305,7 +354,7 @@ RA_HD void q_iter_init(QIter& it, const RingDesc& rd, int64_t k_first, const int
   it.win_base = 0;
   it.k_seg_min = 0;
   it.k_seg_max = 0;
-  if (use_seg) {
+  if (use_seg && RA_IN_RANGE(k_first / kTile, rd.ntiles, kSiteIterMeta)) {
     int4 m = load_meta(meta_b + k_first / kTile);
     it.k_seg_min = m.x;
     it.k_seg_max = m.y;
@@ -313,6 +362,7 @@ RA_HD void q_iter_init(QIter& it, const RingDesc& rd, int64_t k_first, const int
 }
 
 RA_HD bool q_tile_visible(const QIter& it, int32_t q) {
+  if (!RA_IN_RANGE(q, it.nqt, kSiteIterMeta)) return false;
   const int4 m = load_meta(it.meta + (int64_t)q * kQTileBwd / kTile);
   return !(m.y < it.k_seg_min || m.x > it.k_seg_max);
 }

@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
+#include "ra_common.cuh"
 
 namespace ra {
 
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(192, 1)
           }
           pk[e >> 1] = pack_bf16x2(a0, a1);
         }
-        if (valid && n0 + c < p.N) {
+        if (valid && n0 + c < p.N && RA_IN_RANGE(n0 + c + 31, p.N, kSiteFfnOut)) {
           uint4* d4 = reinterpret_cast<uint4*>(dst + n0 + c);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) d4[q4] = make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);

@@ -128,14 +128,17 @@ template <>
 struct FwdTiles<false> {
   KvIter it;
   const int4* meta_b;
+  int32_t ntiles;
   __device__ __forceinline__ void init(const FwdParams& p, int, int64_t q0, const int4* mb, bool use_seg,
                                        bool use_bias) {
     meta_b = mb;
+    ntiles = p.rd.ntiles;
     kv_iter_init(it, p.rd, q0, q0 + 2 * kTile - 1, mb, use_seg, use_bias);
   }
   __device__ __forceinline__ int32_t next(const FwdParams& p) { return kv_iter_next_warp(it, p.rd); }
   __device__ __forceinline__ int4 meta(int32_t t) const {
-    return meta_b ? load_meta(meta_b + t) : make_int4(0, 0, kMetaAnyFinite | kMetaAllZero, 0);
+    return meta_b && RA_IN_RANGE(t, ntiles, kSiteFwdTileMeta) ? load_meta(meta_b + t)
+                                                              : make_int4(0, 0, kMetaAnyFinite | kMetaAllZero, 0);
   }
 };
 
@@ -177,6 +180,7 @@ __global__ void __launch_bounds__(384, 1)
   const int64_t q0 = (int64_t)pair * 2 * kTile;
   const int64_t S = p.rd.S;                   // query rows (Sq in ring-step mode)
   const int64_t Sk = STEP ? p.Sk : S;         // key rows
+  if (!(RA_IN_RANGE(b, p.B, kSiteFwdUnit) && RA_IN_RANGE(h, p.H, kSiteFwdUnit))) return;   // debug build only
 
   auto bar = [&](int i) -> uint32_t { return sbase + L::OFF_BAR + 8u * i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::OFF_MISC);
@@ -358,7 +362,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS_row = tmem + lane_off + (qt ? L::COL_S1 : L::COL_S0);
     const uint32_t tO_row = tmem + lane_off + (qt ? L::COL_O1 : L::COL_O0);
     const int64_t qrow_c = qrow < S ? qrow : S - 1;
-    const int my_seg = use_seg ? p.seg[b * p.seg_sb + qrow_c * p.seg_ss] : 0;
+    const int my_seg = use_seg && RA_IN_RANGE(qrow_c, S, kSiteFwdQuerySeg) ? p.seg[b * p.seg_sb + qrow_c * p.seg_ss] : 0;
     // key-side segment ids (the visiting block's in ring-step mode)
     const int32_t* segk = STEP ? p.seg_k : p.seg;
     const int64_t segk_sb = STEP ? p.segk_sb : p.seg_sb, segk_ss = STEP ? p.segk_ss : p.seg_ss;
@@ -418,7 +422,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int c = c0; c < c0 + 32; ++c) {
             const int64_t j = k0 + c < Sk ? k0 + c : Sk - 1;
-            x[c] = fmaf(x[c], p.scale_log2, __ldg(bp + j * p.bias_ss) * kLog2e);
+            const float bj = RA_IN_RANGE(j, Sk, kSiteFwdKeyBias) ? __ldg(bp + j * p.bias_ss) : 0.f;
+            x[c] = fmaf(x[c], p.scale_log2, bj * kLog2e);
           }
           asm volatile("" ::: "memory");
         }
@@ -444,7 +449,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
               const int64_t j = k0 + 32 * w + c < Sk ? k0 + 32 * w + c : Sk - 1;
-              bits |= (uint32_t)(__ldg(sp + j * segk_ss) == my_seg) << c;
+              bits |= (uint32_t)(RA_IN_RANGE(j, Sk, kSiteFwdKeySeg) && __ldg(sp + j * segk_ss) == my_seg) << c;
             }
             vb[w] = bits;
             asm volatile("" ::: "memory");
@@ -530,10 +535,11 @@ __global__ void __launch_bounds__(384, 1)
       // (m in natural-log units, l, o_acc relative to e^m):
       //   m' = max(m, m_blk), o_acc' = e^(m - m') o_acc + e^(m_blk - m') O, l' likewise.
       const int64_t mi = b * p.ml_sb + h * p.ml_sh + qrow_c * p.ml_ss;
-      const float m_in = p.m_state[mi], l_in = p.l_state[mi];
+      const bool row_in = RA_IN_RANGE(qrow_c, S, kSiteFwdStepState);
+      const float m_in = row_in ? p.m_state[mi] : -INFINITY, l_in = row_in ? p.l_state[mi] : 0.f;
       const float m_blk = (n > 0 && m_ref != -INFINITY) ? m_ref * kLn2 : -INFINITY;
       const float m_new = fmaxf(m_in, m_blk);
-      const bool write = qrow < S && ok && m_new != -INFINITY;
+      const bool write = qrow < S && ok && m_new != -INFINITY && row_in;
       const float a_in = m_in == -INFINITY ? 0.f : expf(m_in - m_new);
       const float a_blk = m_blk == -INFINITY ? 0.f : expf(m_blk - m_new);
       float* ap = p.acc + b * p.acc_sb + qrow_c * p.acc_ss + h * p.acc_sh;
@@ -591,7 +597,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           pkd[e >> 1] = pack_bf16x2(a0, a1);
         }
-        if (qrow < S && ok) {
+        if (qrow < S && ok && RA_IN_RANGE(qrow, S, kSiteFwdOut)) {
           uint4* dst = reinterpret_cast<uint4*>(op + c);
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)

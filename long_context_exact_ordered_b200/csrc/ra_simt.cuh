@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(128) tile_meta_kernel(MaskArgs mk, int64_t S, 
     red[w][0] = smin; red[w][1] = smax; red[w][2] = any_finite; red[w][3] = all_zero;
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && RA_IN_RANGE(t, ntiles, kSiteTileMeta)) {
     for (int i = 1; i < 4; ++i) {
       red[0][0] = min(red[0][0], red[i][0]);
       red[0][1] = max(red[0][1], red[i][1]);
@@ -336,6 +336,7 @@ __global__ void finalize_kernel(const FinalizeArgs a) {
   const int h = (int)(row % a.H);
   const int64_t i = (row / a.H) % a.S;
   const int b = (int)(row / ((int64_t)a.H * a.S));
+  if (!RA_IN_RANGE(b, a.B, kSiteFinalize)) return;
   const int64_t mi = b * a.ml_sb + h * a.ml_sh + i * a.ml_ss;
   const float l = a.l[mi];
   const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -370,6 +371,7 @@ __global__ void lse_merge_kernel(const MergeArgs a) {
   const int h = (int)(row % a.H);
   const int64_t i = (row / a.H) % a.S;
   const int b = (int)(row / ((int64_t)a.H * a.S));
+  if (!RA_IN_RANGE(b, a.B, kSiteFinalize)) return;
   const float xa = a.la[b * a.la_sb + h * a.la_sh + i * a.la_ss];
   const float xb = a.lb[b * a.lb_sb + h * a.lb_sh + i * a.lb_ss];
   const float hi = fmaxf(xa, xb), lo = fminf(xa, xb);
@@ -464,7 +466,7 @@ __global__ void bwd_pre_kernel(const BwdPreArgs a) {
     } else {
       s += static_cast<const float*>(a.o)[io + e] * static_cast<const float*>(a.dO)[id + e];
     }
-    if (a.dqacc) a.dqacc[(bh * a.S + i) * a.D + e] = 0.f;
+    if (a.dqacc && RA_IN_RANGE(bh, (int64_t)a.B * a.H, kSiteBwdPre)) a.dqacc[(bh * a.S + i) * a.D + e] = 0.f;
   }
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) {
@@ -490,6 +492,7 @@ __global__ void dq_convert_kernel(const DqConvertArgs a) {
   const int64_t i = (idx / a.D) % a.S;
   const int64_t bh = idx / ((int64_t)a.D * a.S);
   const int h = (int)(bh % a.H), b = (int)(bh / a.H);
+  if (!RA_IN_RANGE(b, a.B, kSiteDqConvert)) return;
   const float x = a.dqacc[idx];
   const int64_t o = b * a.dq_sb + i * a.dq_ss + h * a.dq_sh + e;
   if (a.bf16) static_cast<__nv_bfloat16*>(a.dq)[o] = __float2bfloat16_rn(x);

@@ -40,11 +40,13 @@ def test_debug_build_exports_its_extra_symbol():
     release build does not carry the debug entry point."""
     dbg = _lib.load_count()
     extra = declared_functions(DEBUG_HEADER)
-    assert extra == ["ra_debug_ex2_rate", "ra_debug_set_counts"]
+    assert extra == ["ra_debug_bounds", "ra_debug_ex2_rate", "ra_debug_set_counts"]
     for n in declared_functions() + extra:
         assert hasattr(dbg, n), n
     assert not hasattr(_lib.load(), "ra_debug_set_counts")
     assert not hasattr(_lib.load(), "ra_debug_ex2_rate")
+    assert not hasattr(_lib.load(), "ra_debug_bounds")
+    assert dbg.ra_debug_bounds(None) == 1
     assert dbg.ra_debug_ex2_rate(0, 1, None, None, None) == 1
     assert dbg.ra_debug_set_counts(None, None) == 0
 
