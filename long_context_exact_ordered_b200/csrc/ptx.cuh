@@ -84,12 +84,17 @@ __device__ __forceinline__ void raise_status(int code) { atomicCAS(&g_ra_status,
 // Bounded wait for completion of phase `parity` of barrier `bar`.  Returns
 // false (and raises the block's abort flag) after `budget` clock cycles or
 // if another role already aborted.
+// Between polls the thread is suspended in hardware (a try_wait with a
+// suspend-time hint) until the phase completes or about kWaitSliceNs pass, so
+// a long wait re-reads the abort flag (a shared-memory load that competes
+// with the tensor cores' operand reads) only once per slice.
+constexpr uint32_t kWaitSliceNs = 20000;
 __device__ __forceinline__ bool ra_wait_budget(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                long long budget) {
   if (mbar_test(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_try_wait_ns(bar, parity, kWaitSliceNs)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > budget) {
       raise_status(9 /* RA_ERR_DEVICE_TIMEOUT */);
@@ -115,7 +120,7 @@ __device__ __forceinline__ bool ra_wait_warp(uint32_t bar, uint32_t parity, vola
 __device__ __forceinline__ bool ra_wait_drain(uint32_t bar, uint32_t parity) {
   if (mbar_test(bar, parity)) return true;
   long long t0 = clock64();
-  while (!mbar_test(bar, parity)) {
+  while (!mbar_try_wait_ns(bar, parity, kWaitSliceNs)) {
     if (clock64() - t0 > RA_SPIN_BUDGET) {
       raise_status(9 /* RA_ERR_DEVICE_TIMEOUT */);
       return false;

@@ -98,6 +98,7 @@ struct BwdLayout {
   static constexpr int THREADS = 512;
   static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
   static_assert(OFF_DQS % 128 == 0, "bulk reduce source alignment");
+  static_assert(OFF_LD % 16 == 0 && LD_BYTES % 16 == 0, "16-byte loads of the LSE / Delta rows");
   static_assert(OFF_ZERO % 1024 == 0 && LBO_DQ % 16 == 0 && (LBO_DQ >> 4) < (1u << 14), "dQ^T operand layout");
   static_assert(D == 64 || D == 128, "head dim");
 };
@@ -148,6 +149,14 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
                : "memory");
 }
 
+// Four floats from shared memory in one access (a warp reading one address
+// gets them as a broadcast: one wavefront for 16 bytes).
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
@@ -391,14 +400,21 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) reg_fence(sr[c]);
         float* x = reinterpret_cast<float*>(sr);
-        const float* nl = reinterpret_cast<const float*>(gbase + L::OFF_LD + st * L::LD_BYTES) + c0;   // -lse*log2e
-        const float* nd = nl + L::QT;                                                                 // -Delta
+        // this group's 32 queries of the stage's -lse*log2e and -Delta rows, read
+        // four at a time (every lane reads the same address)
+        const uint32_t nl = sbase + L::OFF_LD + st * L::LD_BYTES + c0 * 4;
+        const uint32_t nd = nl + L::QT * 4;
         // x = S * log2(e)/sqrt(D) + bias(key) - lse(query) * log2(e), two columns per instruction
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float b0 = nl[c], b1 = nl[c + 1];
-          if (use_bias) fadd2(b0, b1, b0, b1, brow, brow);
+        for (int c = 0; c < 32; c += 4) {
+          const float4 bl = ld_shared_f4(nl + c * 4);
+          float b0 = bl.x, b1 = bl.y, b2 = bl.z, b3 = bl.w;
+          if (use_bias) {
+            fadd2(b0, b1, b0, b1, brow, brow);
+            fadd2(b2, b3, b2, b3, brow, brow);
+          }
           ffma2(x[c], x[c + 1], x[c], x[c + 1], sc, sc, b0, b1);
+          ffma2(x[c + 2], x[c + 3], x[c + 2], x[c + 3], sc, sc, b2, b3);
         }
         // per-element mask on causal-diagonal / ragged / mixed-segment tiles
         const bool need_causal = cbs > 0 && q0 < k_last_blk;
@@ -444,12 +460,17 @@ __global__ void __launch_bounds__(512, 1)
         for (int c = 0; c < 32; ++c) reg_fence(dr[c]);
         uint32_t pp[16], dd[16];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float t0, t1, ds0, ds1;
-          fadd2(t0, t1, __uint_as_float(dr[c]), __uint_as_float(dr[c + 1]), nd[c], nd[c + 1]);   // dP - Delta
+        for (int c = 0; c < 32; c += 4) {
+          const float4 dl = ld_shared_f4(nd + c * 4);
+          float t0, t1, t2, t3, ds0, ds1, ds2, ds3;
+          fadd2(t0, t1, __uint_as_float(dr[c]), __uint_as_float(dr[c + 1]), dl.x, dl.y);   // dP - Delta
+          fadd2(t2, t3, __uint_as_float(dr[c + 2]), __uint_as_float(dr[c + 3]), dl.z, dl.w);
           fmul2(ds0, ds1, pr[c], pr[c + 1], t0, t1);
+          fmul2(ds2, ds3, pr[c + 2], pr[c + 3], t2, t3);
           pp[c >> 1] = pack_bf16x2(pr[c], pr[c + 1]);
+          pp[(c >> 1) + 1] = pack_bf16x2(pr[c + 2], pr[c + 3]);
           dd[c >> 1] = pack_bf16x2(ds0, ds1);
+          dd[(c >> 1) + 1] = pack_bf16x2(ds2, ds3);
         }
         // P^T and dS^T (bf16, two per column) into this slot's first half.
         tmem_st16(slot + L::SLOT_PT + c0, pp);
