@@ -275,3 +275,27 @@ def test_plain_c_client(tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_index_check_sites_match_their_documentation():
+    """The debug build records out-of-range indices by site number
+    (ra_debug_bounds); the header's numbered list of sites must describe the
+    RaSite enumeration of the kernels one to one."""
+    import os
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = open(os.path.join(root, "long_context_exact_ordered_b200", "csrc", "ra_common.cuh")).read()
+    body = src[src.index("enum RaSite : int {"):]
+    body = body[:body.index("};")]
+    names = re.findall(r"\b(kSite\w+)", body)
+    assert names[0] == "kSiteFwdTileMeta" and "= 1," in body.split("\n")[1]
+    assert len(names) == len(set(names))
+    header = open(DEBUG_HEADER).read()
+    listing = header[header.index("Sites:"):header.index("int ra_debug_bounds")]
+    numbers = sorted(int(n) for n in re.findall(r"(?:^|\s)(\d+) (?:forward|backward|ring step|ring-step|tile|dQ|finalize|feed-forward)",
+                                                 listing))
+    assert numbers == list(range(1, len(names) + 1)), (numbers, len(names))
+    for name in names:   # every site is used by some kernel
+        uses = sum(open(os.path.join(root, "long_context_exact_ordered_b200", "csrc", f)).read().count(name)
+                   for f in ("ra_common.cuh", "ra_fwd_sm100.cuh", "ra_bwd_sm100.cuh", "ra_simt.cuh", "ra_ffn_sm100.cuh"))
+        assert uses >= 2, name
