@@ -539,7 +539,9 @@ __global__ void __launch_bounds__(384, 1)
       const float m_in = row_in ? p.m_state[mi] : -INFINITY, l_in = row_in ? p.l_state[mi] : 0.f;
       const float m_blk = (n > 0 && m_ref != -INFINITY) ? m_ref * kLn2 : -INFINITY;
       const float m_new = fmaxf(m_in, m_blk);
-      const bool write = qrow < S && ok && m_new != -INFINITY && row_in;
+      // a block with no visible tile for this CTA leaves the state as it is
+      // (the merge would be the identity), so its rows are not rewritten
+      const bool write = qrow < S && ok && m_new != -INFINITY && row_in && n > 0;
       const float a_in = m_in == -INFINITY ? 0.f : expf(m_in - m_new);
       const float a_blk = m_blk == -INFINITY ? 0.f : expf(m_blk - m_new);
       float* ap = p.acc + b * p.acc_sb + qrow_c * p.acc_ss + h * p.acc_sh;
