@@ -85,6 +85,29 @@ def _hidden(q_start, q_len, k_start, causal_block_size):
     return k_start // c > (q_start + q_len - 1) // c
 
 
+def _segment_ranges(segment_ids, chunks):
+    """Per chunk of this rank ((local start, global start, length) triples),
+    the smallest and largest segment id of every batch row: int64 [chunks, B, 2].
+    An empty chunk gets a range that meets no other."""
+    B = segment_ids.shape[0]
+    out = torch.empty((len(chunks), B, 2), dtype=torch.int64, device=segment_ids.device)
+    for i, (ql, _, qn) in enumerate(chunks):
+        if qn == 0:
+            out[i, :, 0], out[i, :, 1] = 1 << 62, -(1 << 62)
+            continue
+        part = segment_ids[:, ql:ql + qn]
+        out[i, :, 0] = part.amin(dim=1)
+        out[i, :, 1] = part.amax(dim=1)
+    return out
+
+
+def _segments_disjoint(q_range, k_range):
+    """Whether no batch row has a key segment id that also occurs among its
+    queries, judged by their ranges ([B, 2] each): a step over such a pair of
+    chunks would leave the running state unchanged."""
+    return bool(((q_range[:, 1] < k_range[:, 0]) | (q_range[:, 0] > k_range[:, 1])).all())
+
+
 class _Exchange:
     """The ring's double-buffered key/value exchange: send the held block to
     rank+1, receive the next one from rank-1."""
@@ -156,6 +179,19 @@ def ring_attention_forward(q, k, v, attention_bias=None, segment_ids=None, causa
     held = [x.contiguous() for x in [k, v] + ([attention_bias] if attention_bias is not None else []) + (
         [segment_ids] if segment_ids is not None else [])]
     ex = _Exchange(held, group, comm_stream) if world > 1 else None
+    # With segment ids, every rank learns every chunk's segment range once (one
+    # all-gather of a few integers), so that steps over a (query chunk, key
+    # chunk) pair with disjoint segments are skipped on the host, like the
+    # pairs causal masking hides.
+    seg_ranges = None
+    if segment_ids is not None:
+        mine_r = _segment_ranges(segment_ids, chunks)
+        if world > 1:
+            parts = [torch.empty_like(mine_r) for _ in range(world)]
+            dist.all_gather(parts, mine_r, group=group)
+            seg_ranges = [x.cpu() for x in parts]
+        else:
+            seg_ranges = [mine_r.cpu()]
     for t in range(world):
         cur = ex.held(t) if ex else held
         if ex and t < world - 1:
@@ -164,10 +200,12 @@ def ring_attention_forward(q, k, v, attention_bias=None, segment_ids=None, causa
         kc, vc = cur[0], cur[1]
         bias_c = cur[2] if attention_bias is not None else None
         seg_c = cur[-1] if segment_ids is not None else None
-        for (ql, qg, qn), (acc, m, l) in zip(chunks, states):
+        for qi, ((ql, qg, qn), (acc, m, l)) in enumerate(zip(chunks, states)):
             seg_q = None if segment_ids is None else segment_ids[:, ql:ql + qn].contiguous()
-            for kl, kg, kn in chunk_layout(src, world, s_local, layout):
+            for ki, (kl, kg, kn) in enumerate(chunk_layout(src, world, s_local, layout)):
                 if _hidden(qg, qn, kg, causal_block_size):
+                    continue
+                if seg_ranges is not None and _segments_disjoint(seg_ranges[rank][qi], seg_ranges[src][ki]):
                     continue
                 step(q[:, ql:ql + qn], kc[:, kl:kl + kn], vc[:, kl:kl + kn], qg, kg, acc, m, l,
                      bias_blk=None if bias_c is None else bias_c[:, kl:kl + kn].contiguous(),

@@ -62,8 +62,23 @@ def _worker(rank, world, port, cases, errors):
             sh = lambda x: None if x is None else ring.shard(x, rank, world, layout)
             mine = [sh(x) for x in (q, k, v, bb, seg)]
             kept = [None if x is None else x.clone() for x in mine]
-            o, lse = ring.ring_attention_forward(*mine, causal_block_size=c, layout=layout, step=_oracle_step,
+            calls = []
+
+            def counted_step(*a, **kw):
+                calls.append(1)
+                return _oracle_step(*a, **kw)
+
+            o, lse = ring.ring_attention_forward(*mine, causal_block_size=c, layout=layout, step=counted_step,
                                                  finalize=_oracle_finalize)
+            if segments:
+                # the same ring without segment ids makes every step the mask allows
+                plain = []
+                ring.ring_attention_forward(*mine[:4], None, causal_block_size=c, layout=layout,
+                                            step=lambda *a, **kw: (plain.append(1), _oracle_step(*a, **kw))[1],
+                                            finalize=_oracle_finalize)
+                if not len(calls) < len(plain):
+                    errors.put(f"rank {rank} {layout}: no step skipped for disjoint segments "
+                               f"({len(calls)} vs {len(plain)})")
             if any(a is not None and not torch.equal(a, b) for a, b in zip(mine, kept)):
                 errors.put(f"rank {rank} {layout}: the caller's tensors were modified")
             want_o = ring.shard(torch.from_numpy(ro), rank, world, layout)
