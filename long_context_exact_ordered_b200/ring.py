@@ -165,7 +165,8 @@ def ring_attention_forward(q, k, v, attention_bias=None, segment_ids=None, causa
     None; segment_ids: int32 [B, S_local] or None (this rank's keys and
     queries).  Returns (o [B, S_local, H, D], lse fp32 [B, H, S_local]) for
     this rank's queries, in local order.  Every rank of ``group`` must call
-    it with the same shapes.  ``step`` / ``finalize`` default to the
+    it with the same shapes, and all with segment ids or all without: with
+    them, the ranks first all-gather their chunks' segment ranges.  ``step`` / ``finalize`` default to the
     library's ``ring_step`` / ``finalize``; the CPU tests pass the oracle's
     here to check the exchange protocol without a GPU.
     """

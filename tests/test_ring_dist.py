@@ -1,6 +1,6 @@
 """The cross-rank ring (long_context_exact_ordered_b200.ring) on CPU processes.
 
-World sizes 2 and 3 over gloo: every rank holds its shard of the sequence,
+World sizes 2, 3 and 4 over gloo: every rank holds its shard of the sequence,
 key/value blocks (with their segment ids and bias) travel round the ring
 through torch.distributed point-to-point exchanges, and the per-step
 arithmetic is the oracle's online-softmax step in float64 (passed in as the
@@ -103,7 +103,7 @@ CASES = [("zigzag", 1, False, False), ("contiguous", 1, False, False), ("zigzag"
          ("zigzag", 3, True, False), ("contiguous", 1, False, True)]
 
 
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 4])
 def test_ring_across_ranks_equals_full_attention(world):
     ctx = mp.get_context("spawn")
     errors = ctx.SimpleQueue()
